@@ -1,0 +1,11 @@
+"""CPU fp64 oracle for NABLA block-sparse video attention.
+
+TEST INFRASTRUCTURE ONLY: the reference the CUDA path is checked against.
+Only the tests, the smoke check and the benchmark's CPU-baseline leg may
+import it; the library never does, and the two share no code.
+"""
+from .nabla import (  # noqa: F401
+    widen_bf16, fractal_order, flatten, unflatten, pool, reduced_map, cdf_keep,
+    block_coords, sta_keep, pooled_head, nabla_mask, masked_attention,
+    attention_head, nabla_attention,
+)

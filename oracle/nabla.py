@@ -1,0 +1,220 @@
+"""Plain fp64 CPU oracle for NABLA block-sparse video self-attention.
+
+TEST INFRASTRUCTURE ONLY. The tests, the smoke check and the benchmark's
+CPU-baseline leg are the only callers; the CUDA library never imports it and
+shares no code with it.
+
+Every function follows the method as described on the page
+"NABLA - Neighborhood Adaptive Block-Level Attention per la Generazione
+Efficiente di Video" (gist.science/it/paper/2507.13546), section
+"Metodologia: NABLA", and is written for a reader to check by eye: fp64
+throughout, library primitives (matmul, sort, cumsum) as single steps, no
+blocking, fusion or reordering beyond what the method states.
+
+Readings taken where the page is silent (each one is listed in the design
+notes as well):
+
+* Fractal order: time outermost, then patch row, then patch column; inside a
+  P x P patch the tokens are row-major (h % P, then w % P).
+* Pooling "in N x N blocks" means the mean of N consecutive tokens of the
+  reordered sequence; the N x N refers to the block of the attention map.
+* The reduced map uses the same 1/sqrt(d) scale as the main attention and no
+  causal mask.
+* CDF thresholding keeps the shortest prefix of the row, sorted by descending
+  probability (ties: smaller block index first), whose mass reaches 1 - thr:
+  block j is kept iff the mass strictly before it is < 1 - thr. thr = 0 is
+  defined as dense.
+* The STA window is centred on the query block in block units, clipped at the
+  grid edges; window sizes are odd; (0, 0, 0) means no STA.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def widen_bf16(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns (uint16) -> exact float64 values."""
+    u32 = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return u32.view(np.float32).astype(np.float64)
+
+
+# --- Metodologia 1: "Riordinamento dei Token (Fractal Flattening)" ----------
+
+def fractal_order(T: int, Hh: int, Ww: int, P: int) -> np.ndarray:
+    """perm[i] = natural-order index of the token at position i of the
+    fractally flattened sequence.
+
+    Tokens of each P x P spatial patch become contiguous; frames stay in
+    time order. Natural order index of (t, h, w) is t*Hh*Ww + h*Ww + w.
+    Position order is (t, patch row hp, patch column wp, h % P, w % P).
+    """
+    if Hh % P or Ww % P:
+        raise ValueError("Hh and Ww must be multiples of P")
+    t = np.arange(T).reshape(T, 1, 1, 1, 1)
+    hp = np.arange(Hh // P).reshape(1, Hh // P, 1, 1, 1)
+    wp = np.arange(Ww // P).reshape(1, 1, Ww // P, 1, 1)
+    hi = np.arange(P).reshape(1, 1, 1, P, 1)
+    wi = np.arange(P).reshape(1, 1, 1, 1, P)
+    natural = t * (Hh * Ww) + (hp * P + hi) * Ww + (wp * P + wi)
+    return natural.reshape(-1).astype(np.int64)
+
+
+def flatten(x: np.ndarray, perm: np.ndarray) -> np.ndarray:
+    """Reorder tokens (axis -2) from natural order into fractal order."""
+    return x[..., perm, :]
+
+
+def unflatten(xp: np.ndarray, perm: np.ndarray) -> np.ndarray:
+    """Inverse of ``flatten``: scatter fractal-order rows back to natural order."""
+    out = np.empty_like(xp)
+    out[..., perm, :] = xp
+    return out
+
+
+# --- Metodologia 2: "Costruzione della Maschera Adattiva" -------------------
+
+def pool(xp: np.ndarray, N: int) -> np.ndarray:
+    """Sottocampionamento: mean of each run of N consecutive reordered tokens.
+
+    [..., S, d] -> [..., S/N, d].
+    """
+    S, d = xp.shape[-2], xp.shape[-1]
+    if S % N:
+        raise ValueError("S must be a multiple of N")
+    return xp.reshape(xp.shape[:-2] + (S // N, N, d)).mean(axis=-2)
+
+
+def reduced_map(qbar: np.ndarray, kbar: np.ndarray) -> np.ndarray:
+    """Attenzione Ridotta: full softmax(Qbar Kbar^T / sqrt(d)) between pooled
+    blocks, row-wise, computed with max subtraction. [..., nb, nb]."""
+    d = qbar.shape[-1]
+    logits = qbar @ np.swapaxes(kbar, -1, -2) / np.sqrt(d)
+    e = np.exp(logits - logits.max(axis=-1, keepdims=True))
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def cdf_keep(A: np.ndarray, thr: float) -> np.ndarray:
+    """CDF Thresholding: per row, keep the smallest set of blocks, taken in
+    order of descending probability, whose cumulative mass reaches 1 - thr.
+
+    Block j is kept iff the mass of the blocks before it in that order is
+    strictly below 1 - thr (so the first block is always kept). Equal
+    probabilities are ordered by ascending block index. thr = 0 keeps all.
+    """
+    if not 0.0 <= thr < 1.0:
+        raise ValueError("thr must lie in [0, 1)")
+    if thr == 0.0:
+        return np.ones(A.shape, dtype=bool)
+    order = np.argsort(-A, axis=-1, kind="stable")
+    a_sorted = np.take_along_axis(A, order, axis=-1)
+    incl = np.cumsum(a_sorted, axis=-1)
+    before = np.concatenate([np.zeros(A.shape[:-1] + (1,)), incl[..., :-1]], axis=-1)
+    keep_sorted = before < (1.0 - thr)
+    keep = np.empty(A.shape, dtype=bool)
+    np.put_along_axis(keep, order, keep_sorted, axis=-1)
+    return keep
+
+
+def block_coords(T: int, Hh: int, Ww: int, P: int) -> np.ndarray:
+    """(t, hp, wp) of every block in fractal order when N = P*P, shape [nb, 3]."""
+    nh, nw = Hh // P, Ww // P
+    b = np.arange(T * nh * nw)
+    return np.stack([b // (nh * nw), (b // nw) % nh, b % nw], axis=1)
+
+
+# --- Metodologia 3: "Integrazione Ibrida con STA" ---------------------------
+
+def sta_keep(T: int, Hh: int, Ww: int, P: int, sta) -> np.ndarray:
+    """Static sliding-tile window in block units: q-block and k-block are
+    paired iff their distance along each of (t, hp, wp) is at most half the
+    (odd) window size. (0, 0, 0) is no window. [nb, nb] bool."""
+    st, sh, sw = sta
+    c = block_coords(T, Hh, Ww, P)
+    nb = c.shape[0]
+    if (st, sh, sw) == (0, 0, 0):
+        return np.zeros((nb, nb), dtype=bool)
+    if min(st, sh, sw) < 1 or not (st % 2 and sh % 2 and sw % 2):
+        raise ValueError("STA window sizes must be odd and positive")
+    diff = np.abs(c[:, None, :] - c[None, :, :])
+    return ((diff[..., 0] <= st // 2) & (diff[..., 1] <= sh // 2)
+            & (diff[..., 2] <= sw // 2))
+
+
+def _as_f64(x):
+    return widen_bf16(x) if np.asarray(x).dtype == np.uint16 else np.asarray(x, dtype=np.float64)
+
+
+def pooled_head(x, T, Hh, Ww, P, N):
+    """Pooled blocks of one head: natural-order [S, d] -> [nb, d] float64."""
+    return pool(flatten(_as_f64(x), fractal_order(T, Hh, Ww, P)), N)
+
+
+def nabla_mask(q, k, T, Hh, Ww, P, N, thr, sta):
+    """The final block mask M = M_nabla OR M_STA for every (batch, head).
+
+    q, k: natural-order [BH, S, d] (bf16 bits as uint16, or floats), handled
+    one head at a time. Returns (M, M_nabla, A): bool [BH, nb, nb] masks and
+    the float64 reduced map.
+    """
+    if N != P * P:
+        raise ValueError("this reading needs N == P*P (one block = one patch)")
+    m_sta = sta_keep(T, Hh, Ww, P, sta)
+    BH, nb = q.shape[0], q.shape[1] // N
+    A = np.empty((BH, nb, nb))
+    m_nabla = np.empty((BH, nb, nb), dtype=bool)
+    for bh in range(BH):
+        A[bh] = reduced_map(pooled_head(q[bh], T, Hh, Ww, P, N),
+                            pooled_head(k[bh], T, Hh, Ww, P, N))
+        m_nabla[bh] = cdf_keep(A[bh], thr)
+    return m_nabla | m_sta[None], m_nabla, A
+
+
+# --- Espansione + masked exact attention ------------------------------------
+
+def masked_attention(qp, kp, vp, mask, N, rows=None):
+    """Exact attention in fractal order with every dropped N x N block at -inf.
+
+    qp, kp, vp: [S, d] float64 (one head, fractal order); mask: [nb, nb] bool.
+    rows: fractal-order query positions to compute (default: all).
+    Returns [len(rows), d] float64.
+    """
+    S, d = qp.shape
+    rows = np.arange(S) if rows is None else np.asarray(rows)
+    out = np.empty((rows.size, vp.shape[-1]))
+    qb_of_row = rows // N
+    for qb in np.unique(qb_of_row):
+        sel = np.nonzero(qb_of_row == qb)[0]
+        kept_blocks = np.nonzero(mask[qb])[0]
+        cols = (kept_blocks[:, None] * N + np.arange(N)[None, :]).reshape(-1)
+        s = qp[rows[sel]] @ kp[cols].T / np.sqrt(d)
+        e = np.exp(s - s.max(axis=-1, keepdims=True))
+        out[sel] = (e / e.sum(axis=-1, keepdims=True)) @ vp[cols]
+    return out
+
+
+def attention_head(q, k, v, T, Hh, Ww, P, N, mask, tokens=None):
+    """One head of the whole path: fractal flatten, masked attention over the
+    kept blocks of ``mask`` [nb, nb], inverse flatten.
+
+    q, k, v: natural-order [S, d]. tokens: natural-order query indices to
+    compute (default all); each output row is exact on its own, so a sample
+    of rows equals the same rows of the full result. Returns [n, d] float64.
+    """
+    perm = fractal_order(T, Hh, Ww, P)
+    qp, kp, vp = (flatten(_as_f64(x), perm) for x in (q, k, v))
+    if tokens is None:
+        return unflatten(masked_attention(qp, kp, vp, mask, N), perm)
+    pos_of = np.empty_like(perm)
+    pos_of[perm] = np.arange(perm.size)
+    return masked_attention(qp, kp, vp, mask, N, rows=pos_of[np.asarray(tokens)])
+
+
+def nabla_attention(q, k, v, T, Hh, Ww, P, N, thr, sta, mask=None):
+    """Whole path for natural-order [BH, S, d] inputs: mask build (unless
+    ``mask`` [BH, nb, nb] is given) then per-head masked attention.
+    Returns (O natural order float64 [BH, S, d], mask)."""
+    if mask is None:
+        mask, _, _ = nabla_mask(q, k, T, Hh, Ww, P, N, thr, sta)
+    out = np.stack([attention_head(q[bh], k[bh], v[bh], T, Hh, Ww, P, N, mask[bh])
+                    for bh in range(q.shape[0])])
+    return out, mask
