@@ -1,0 +1,351 @@
+"""Benchmark of the block-sparse video attention path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-cpu-baseline]
+
+One step = one pass of the whole hot path over one batch: sparse_attn_plan
+(block pooling, reduced map, CDF threshold, STA union, block lists) followed by
+sparse_attn_fwd (block-sparse attention over the kept pairs, written back in
+natural token order). The metric is attention TFLOP/s counted on kept blocks
+only (4 * 64^2 * d per kept (q-block, k-block) pair), whole step; the JSON
+also carries the mask-build time, the attention kernel's own TFLOP/s and its
+fraction of the measured bf16 tensor peak.
+
+With N > 1 (launched by torch.distributed.run) every rank runs its own copy of
+the workload (heads are independent: weak scaling, no data-path collective);
+the time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded
+sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from dynamic_block_sparse_fractal_b200 import workloads as W  # noqa: E402
+
+METRIC = "sparse attn TFLOP/s on kept blocks + mask-build µs; % of BF16 tensor peak"
+UNIT = "TFLOP/s"
+DEFAULT_WORKLOAD = W.HUNYUAN
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def pick_workload(name):
+    if name is None:
+        return DEFAULT_WORKLOAD
+    if name in W.WORKLOADS:
+        return W.WORKLOADS[name]
+    if name.startswith("sweep:"):
+        return W.sweep(int(name.split(":")[1]))
+    raise SystemExit(f"unknown workload {name}; choose from {sorted(W.WORKLOADS)} or sweep:K")
+
+
+def kept_flops_per_pair(w):
+    return 4.0 * w.N * w.N * w.d
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def to_device(bits, w, device):
+    import torch
+    t = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+    return t.reshape(w.B, w.H, w.S, w.d).to(device)
+
+
+def run_ours(args, w, rank, world):
+    import torch
+    from dynamic_block_sparse_fractal_b200 import api
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    q_h, k_h, v_h = W.make_inputs(w)
+    q, k, v = (to_device(x, w, dev) for x in (q_h, k_h, v_h))
+    desc = api.desc_for(w)
+    ws = api.alloc_workspace(desc, dev)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(args.warmup):
+        api.plan(desc, q, k, ws)
+        api.fwd(desc, q, k, v, ws, out)
+    st = api.check(desc, ws)
+    if st != api.SA_OK:
+        raise SystemExit(f"device status after warm-up: {api.status_string(st)}")
+
+    views = api.get_mask(desc, ws)
+    kept_pairs = int(views["cnt"].sum().item())
+    union_entries = int(views["tile_cnt"].sum().item())
+    kept_flops = kept_pairs * kept_flops_per_pair(w)
+    computed_flops = union_entries * 2 * kept_flops_per_pair(w)  # 128-row tiles
+    sparsity = 1.0 - kept_pairs / (w.BH * w.nb * w.nb)
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            api.plan(desc, q, k, ws)
+            ev[i][1].record(stream)
+            api.fwd(desc, q, k, v, ws, out)
+            ev[i][2].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    total_ms = t0.elapsed_time(t1)
+    plan_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    fwd_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    st = api.check(desc, ws)
+    if st != api.SA_OK:
+        raise SystemExit(f"device status after timing: {api.status_string(st)}")
+    if dist is not None:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    # ---- end to end through the public API, host buffers, copies timed
+    pin = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).reshape(w.B, w.H, w.S, w.d)
+           .pin_memory() for x in (q_h, k_h, v_h)]
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    e2e_steps = max(1, min(args.steps, 5))
+    attn = api.NablaAttention(w.B, w.H, w.T, w.Hh, w.Ww, w.d, w.thr, w.sta, device=dev)
+
+    def e2e_step():
+        qd = pin[0].to(dev, non_blocking=True)
+        kd = pin[1].to(dev, non_blocking=True)
+        vd = pin[2].to(dev, non_blocking=True)
+        o = attn(qd, kd, vd)
+        out_h.copy_(o, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    a0 = torch.cuda.Event(enable_timing=True)
+    a1 = torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    a1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = a0.elapsed_time(a1) / e2e_steps
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    st = attn.check()
+    if st != api.SA_OK:
+        raise SystemExit(f"device status after e2e: {api.status_string(st)}")
+
+    peaks, src = load_peaks()
+    ms_step = total_ms / args.steps
+    fwd_avg = statistics.mean(fwd_ms)
+    attn_tflops = kept_flops / (fwd_avg * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    line = {
+        "metric": METRIC, "value": round(world * kept_flops / (ms_step * 1e-3) / 1e12, 2),
+        "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {**w.describe(), "per_gpu": "one full copy of the workload per GPU",
+                   "l2": "inputs larger than L2 (3 x %.0f MB bf16)" % (w.BH * w.S * w.d * 2 / 1e6)},
+        "mask_build_us": round(statistics.mean(plan_ms) * 1e3, 1),
+        "attn_fwd_ms": round(fwd_avg, 4),
+        "attn_kept_tflops": round(attn_tflops, 2),
+        "pct_bf16_peak": round(100.0 * attn_tflops / peak, 2),
+        "sparsity": round(sparsity, 4),
+        "kept_pairs": kept_pairs,
+        "computed_over_kept": round(computed_flops / kept_flops, 4),
+        "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 2), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(attn_tflops / peak, 4),
+                     "traffic": None, "kernel": "sa::attn_kernel<128>",
+                     "peak_source": f"{src} bf16 burst"},
+        "e2e": {"value": round(world * kept_flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+                "ms_per_step": round(e2e_ms, 3),
+                "h2d_bytes_per_step": int(3 * q.numel() * 2),
+                "d2h_bytes_per_step": int(out.numel() * out.element_size())},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return line
+
+
+def oracle_sample(w, budget_s=20.0, seed=0):
+    """Times the fp64 oracle on a bounded sample of workload w.
+
+    Sample: heads 0..h-1 in full for the mask build (pool, reduced map, CDF,
+    STA), then exact masked attention for whole q-blocks drawn at random from
+    those heads until the time budget is spent. Returns kept-block TFLOP/s of
+    the attention part, the mask-build seconds per head and a description."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        cores = 1
+    heads = [0]
+    q, k, v = W.make_inputs(w, heads=range(0, 1))
+    t = time.perf_counter()
+    M, _, _ = oracle.nabla_mask(q, k, w.T, w.Hh, w.Ww, w.P, w.N, w.thr, w.sta)
+    mask_s = time.perf_counter() - t
+    rng = np.random.default_rng(seed)
+    order = rng.permutation(w.nb)
+    perm = oracle.fractal_order(w.T, w.Hh, w.Ww, w.P)
+    qp, kp, vp = (oracle.flatten(oracle.widen_bf16(x[0]), perm) for x in (q, k, v))
+    pairs, spent, nq = 0, 0.0, 0
+    t = time.perf_counter()
+    for qb in order:
+        rows = np.arange(qb * w.N, (qb + 1) * w.N)
+        oracle.masked_attention(qp, kp, vp, M[0], w.N, rows=rows)
+        pairs += int(M[0, qb].sum())
+        nq += 1
+        spent = time.perf_counter() - t
+        if spent > budget_s:
+            break
+    tflops = pairs * kept_flops_per_pair(w) / spent / 1e12
+    desc = (f"head 0 of {w.BH}: full mask build ({mask_s:.1f} s), then exact masked attention "
+            f"on {nq} of {w.nb} q-blocks drawn at random ({spent:.1f} s); value = kept-block "
+            f"TFLOP/s of that attention")
+    return tflops, mask_s, cores, desc
+
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return None
+    vals = []
+    budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for i in range(args.warmup + args.steps):
+        tf, mask_s, cores, desc = oracle_sample(w, budget_s=budget, seed=i)
+        if i >= args.warmup:
+            vals.append(tf)
+    value = statistics.mean(vals)
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": w.describe(),
+        "cpu_baseline": {"kind": "oracle", "cores": cores, "sample": desc, "value": value,
+                         "unit": UNIT},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    w = pick_workload(args.workload)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", str(args.gpus if args.gpus == 1 else 1)))
+    if args.impl == "reference":
+        line = run_reference(args, w, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    line = run_ours(args, w, rank, world)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            tf, mask_s, cores, desc = oracle_sample(w, budget_s=15.0)
+            line["cpu_baseline"] = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                    "sample": desc, "mask_build_s_per_head": round(mask_s, 2)}
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

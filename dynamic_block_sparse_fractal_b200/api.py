@@ -1,0 +1,219 @@
+"""Python binding of libsparse_attn.so (include/sparse_attn.h).
+
+Argument marshalling only: every step of the attention path runs in the
+library's CUDA kernels. PyTorch provides device memory and streams. If the
+library has not been built, every call raises; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libsparse_attn.so")
+
+SA_OK = 0
+SA_ERR_INVALID_ARG = 1
+SA_ERR_UNSUPPORTED = 2
+SA_ERR_WORKSPACE = 3
+SA_ERR_CUDA = 4
+SA_ERR_DEVICE_TIMEOUT = 5
+SA_DEBUG_STALL_LOADER = 1
+
+SYMBOLS = (
+    "sparse_attn_workspace_size", "sparse_attn_plan", "sparse_attn_fwd",
+    "sparse_attn_permute", "sparse_attn_get_mask", "sparse_attn_tile_blocks",
+    "sparse_attn_check", "sparse_attn_status_string",
+)
+
+
+class SaDesc(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int),
+                ("Hh", ctypes.c_int), ("Ww", ctypes.c_int), ("d", ctypes.c_int),
+                ("N", ctypes.c_int), ("P", ctypes.c_int), ("thr", ctypes.c_float),
+                ("sta_t", ctypes.c_int), ("sta_h", ctypes.c_int), ("sta_w", ctypes.c_int),
+                ("out_fp32", ctypes.c_int), ("debug_flags", ctypes.c_int)]
+
+
+class SaMaskViews(ctypes.Structure):
+    _fields_ = [("qbar", ctypes.c_void_p), ("kbar", ctypes.c_void_p), ("cnt", ctypes.c_void_p),
+                ("idx", ctypes.c_void_p), ("tile_cnt", ctypes.c_void_p),
+                ("tile_idx", ctypes.c_void_p), ("nb", ctypes.c_int), ("ntile", ctypes.c_int)]
+
+
+class SparseAttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing; build it with "
+                "`python -m dynamic_block_sparse_fractal_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, sz, i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+        dp = ctypes.POINTER(SaDesc)
+        L.sparse_attn_workspace_size.argtypes = [dp, ctypes.POINTER(sz)]
+        L.sparse_attn_plan.argtypes = [dp, vp, vp, vp, sz, vp]
+        L.sparse_attn_fwd.argtypes = [dp, vp, vp, vp, vp, sz, vp, vp]
+        L.sparse_attn_permute.argtypes = [dp, vp, vp, i32, vp]
+        L.sparse_attn_get_mask.argtypes = [dp, vp, sz, ctypes.POINTER(SaMaskViews)]
+        L.sparse_attn_tile_blocks.argtypes = [dp, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)]
+        L.sparse_attn_check.argtypes = [dp, vp, sz, vp]
+        L.sparse_attn_status_string.argtypes = [i32]
+        L.sparse_attn_status_string.restype = ctypes.c_char_p
+        for name in SYMBOLS[:-1]:
+            getattr(L, name).restype = i32
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().sparse_attn_status_string(int(status)).decode()
+
+
+def _ok(status: int, what: str) -> None:
+    if status != SA_OK:
+        raise SparseAttnError(status, what)
+
+
+def make_desc(B: int, H: int, T: int, Hh: int, Ww: int, d: int, thr: float,
+              sta=(0, 0, 0), N: int = 64, P: int = 8, out_fp32: bool = False,
+              debug_flags: int = 0) -> SaDesc:
+    return SaDesc(B, H, T, Hh, Ww, d, N, P, float(thr), int(sta[0]), int(sta[1]), int(sta[2]),
+                  int(bool(out_fp32)), int(debug_flags))
+
+
+def desc_for(w, out_fp32: bool = False, debug_flags: int = 0) -> SaDesc:
+    """Descriptor of a workload from ``workloads``."""
+    return make_desc(w.B, w.H, w.T, w.Hh, w.Ww, w.d, w.thr, w.sta, w.N, w.P, out_fp32,
+                     debug_flags)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _ptr(t: Optional[torch.Tensor]) -> ctypes.c_void_p:
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _check_qkv(desc: SaDesc, *ts: torch.Tensor) -> None:
+    S = desc.T * desc.Hh * desc.Ww
+    for t in ts:
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous bf16 CUDA tensors")
+        if tuple(t.shape) != (desc.B, desc.H, S, desc.d):
+            raise ValueError(f"expected shape {(desc.B, desc.H, S, desc.d)}, got {tuple(t.shape)}")
+
+
+def workspace_size(desc: SaDesc) -> int:
+    n = ctypes.c_size_t(0)
+    _ok(lib().sparse_attn_workspace_size(ctypes.byref(desc), ctypes.byref(n)), "workspace_size")
+    return n.value
+
+
+def alloc_workspace(desc: SaDesc, device=None) -> torch.Tensor:
+    return torch.empty(workspace_size(desc), dtype=torch.uint8,
+                       device=device if device is not None else "cuda")
+
+
+def plan(desc: SaDesc, q: torch.Tensor, k: torch.Tensor, workspace: torch.Tensor,
+         stream=None) -> None:
+    _check_qkv(desc, q, k)
+    _ok(lib().sparse_attn_plan(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(workspace),
+                               workspace.numel(), _stream(stream)), "plan")
+
+
+def fwd(desc: SaDesc, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+        workspace: torch.Tensor, out: torch.Tensor, stream=None) -> torch.Tensor:
+    _check_qkv(desc, q, k, v)
+    want = torch.float32 if desc.out_fp32 else torch.bfloat16
+    if out.dtype != want or out.shape != q.shape or not out.is_contiguous():
+        raise ValueError(f"out must be a contiguous {want} tensor shaped like q")
+    _ok(lib().sparse_attn_fwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(workspace),
+                              workspace.numel(), _ptr(out), _stream(stream)), "fwd")
+    return out
+
+
+def permute(desc: SaDesc, x: torch.Tensor, y: torch.Tensor, inverse: bool = False,
+            stream=None) -> torch.Tensor:
+    _check_qkv(desc, x, y)
+    _ok(lib().sparse_attn_permute(ctypes.byref(desc), _ptr(x), _ptr(y), int(inverse),
+                                  _stream(stream)), "permute")
+    return y
+
+
+def check(desc: SaDesc, workspace: torch.Tensor, stream=None) -> int:
+    """Synchronises the stream; returns the status (SA_OK or an error code)."""
+    return lib().sparse_attn_check(ctypes.byref(desc), _ptr(workspace), workspace.numel(),
+                                   _stream(stream))
+
+
+def tile_blocks(desc: SaDesc, tile: int) -> Tuple[int, int]:
+    a, b = ctypes.c_int(0), ctypes.c_int(0)
+    _ok(lib().sparse_attn_tile_blocks(ctypes.byref(desc), int(tile), ctypes.byref(a),
+                                      ctypes.byref(b)), "tile_blocks")
+    return a.value, b.value
+
+
+def get_mask(desc: SaDesc, workspace: torch.Tensor) -> dict:
+    """Tensor views (no copies) of the planned lists inside ``workspace``."""
+    v = SaMaskViews()
+    _ok(lib().sparse_attn_get_mask(ctypes.byref(desc), _ptr(workspace), workspace.numel(),
+                                   ctypes.byref(v)), "get_mask")
+    base = workspace.data_ptr()
+    BH, nb, nt, d = desc.B * desc.H, v.nb, v.ntile, desc.d
+
+    def view(ptr, count, dtype, shape):
+        off = ptr - base
+        nbytes = count * torch.tensor([], dtype=dtype).element_size()
+        return workspace[off:off + nbytes].view(dtype).view(*shape)
+
+    return {
+        "nb": nb, "ntile": nt,
+        "qbar": view(v.qbar, BH * nb * d, torch.float32, (BH, nb, d)),
+        "kbar": view(v.kbar, BH * nb * d, torch.float32, (BH, nb, d)),
+        "cnt": view(v.cnt, BH * nb, torch.int32, (BH, nb)),
+        "idx": view(v.idx, BH * nb * nb, torch.int32, (BH, nb, nb)),
+        "tile_cnt": view(v.tile_cnt, BH * nt, torch.int32, (BH, nt)),
+        "tile_idx": view(v.tile_idx, BH * nt * nb, torch.int32, (BH, nt, nb)),
+    }
+
+
+class NablaAttention:
+    """User-facing wrapper: owns a workspace; ``plan`` builds the block mask,
+    ``forward`` runs the block-sparse attention; calling it does both."""
+
+    def __init__(self, B, H, T, Hh, Ww, d, thr, sta=(0, 0, 0), out_fp32=False, device="cuda"):
+        self.desc = make_desc(B, H, T, Hh, Ww, d, thr, sta, out_fp32=out_fp32)
+        self.workspace = alloc_workspace(self.desc, device)
+
+    def plan(self, q, k, stream=None):
+        plan(self.desc, q, k, self.workspace, stream)
+
+    def forward(self, q, k, v, out=None, stream=None):
+        if out is None:
+            out = torch.empty(q.shape, device=q.device,
+                              dtype=torch.float32 if self.desc.out_fp32 else torch.bfloat16)
+        return fwd(self.desc, q, k, v, self.workspace, out, stream)
+
+    def __call__(self, q, k, v, out=None, stream=None):
+        self.plan(q, k, stream)
+        return self.forward(q, k, v, out, stream)
+
+    def check(self, stream=None) -> int:
+        return check(self.desc, self.workspace, stream)

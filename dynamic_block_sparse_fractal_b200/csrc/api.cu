@@ -1,0 +1,209 @@
+// Host side of the C ABI declared in include/sparse_attn.h: argument
+// validation, workspace layout, launch sequencing and status reporting.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "kernels.cuh"
+#include "layout.cuh"
+#include "tma_host.h"
+
+using namespace sa;
+
+namespace {
+
+// Largest block count per head the mask kernel's shared memory can hold
+// (16 rows of fp32 probabilities plus keep bitmaps).
+constexpr int kMaxBlocks = 2880;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+sa_status validate(const sa_desc* d) {
+  if (d == nullptr) return SA_ERR_INVALID_ARG;
+  if (d->B < 1 || d->H < 1 || d->T < 1 || d->Hh < 1 || d->Ww < 1 || d->d < 1 || d->N < 1 ||
+      d->P < 1)
+    return SA_ERR_INVALID_ARG;
+  if (!(d->thr >= 0.0f && d->thr < 1.0f)) return SA_ERR_INVALID_ARG;  // also rejects NaN
+  const bool no_sta = d->sta_t == 0 && d->sta_h == 0 && d->sta_w == 0;
+  if (!no_sta) {
+    if (d->sta_t < 1 || d->sta_h < 1 || d->sta_w < 1) return SA_ERR_INVALID_ARG;
+    if (!(d->sta_t & 1) || !(d->sta_h & 1) || !(d->sta_w & 1)) return SA_ERR_INVALID_ARG;
+  }
+  if (d->out_fp32 != 0 && d->out_fp32 != 1) return SA_ERR_INVALID_ARG;
+  if (d->debug_flags & ~SA_DEBUG_STALL_LOADER) return SA_ERR_INVALID_ARG;
+  if (d->d != 64 && d->d != 128) return SA_ERR_UNSUPPORTED;
+  if (d->P != 8 || d->N != d->P * d->P) return SA_ERR_UNSUPPORTED;
+  if (d->Hh % d->P || d->Ww % d->P) return SA_ERR_UNSUPPORTED;
+  const long long BH = (long long)d->B * d->H;
+  const long long nb = (long long)d->T * (d->Hh / d->P) * (d->Ww / d->P);
+  if (BH > 65535 || nb > kMaxBlocks) return SA_ERR_UNSUPPORTED;
+  return SA_OK;
+}
+
+sa_status check_ws(const Geometry& g, const void* ws, size_t ws_bytes) {
+  if (ws == nullptr || !aligned(ws, 256)) return SA_ERR_INVALID_ARG;
+  if (ws_bytes < make_ws_layout(g).total) return SA_ERR_WORKSPACE;
+  return SA_OK;
+}
+
+sa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SA_OK : SA_ERR_CUDA; }
+
+template <class T>
+T* at(void* base, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(base) + off);
+}
+template <class T>
+const T* at(const void* base, size_t off) {
+  return reinterpret_cast<const T*>(static_cast<const uint8_t*>(base) + off);
+}
+
+}  // namespace
+
+extern "C" {
+
+sa_status sparse_attn_workspace_size(const sa_desc* desc, size_t* bytes) {
+  const sa_status st = validate(desc);
+  if (st != SA_OK) return st;
+  if (bytes == nullptr) return SA_ERR_INVALID_ARG;
+  *bytes = make_ws_layout(make_geometry(*desc)).total;
+  return SA_OK;
+}
+
+sa_status sparse_attn_plan(const sa_desc* desc, const void* q, const void* k, void* workspace,
+                           size_t ws_bytes, void* stream) {
+  sa_status st = validate(desc);
+  if (st != SA_OK) return st;
+  if (q == nullptr || k == nullptr || !aligned(q, 16) || !aligned(k, 16))
+    return SA_ERR_INVALID_ARG;
+  const Geometry g = make_geometry(*desc);
+  st = check_ws(g, workspace, ws_bytes);
+  if (st != SA_OK) return st;
+  const WsLayout w = make_ws_layout(g);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  cudaError_t e = cudaMemsetAsync(at<uint32_t>(workspace, w.status), 0, 256, s);
+  if (e != cudaSuccess) return SA_ERR_CUDA;
+  e = launch_pool(q, k, at<float>(workspace, w.qbar), at<float>(workspace, w.kbar), g, s);
+  if (e != cudaSuccess) return SA_ERR_CUDA;
+
+  MaskArgs m;
+  m.qbar = at<float>(workspace, w.qbar);
+  m.kbar = at<float>(workspace, w.kbar);
+  m.cnt = at<int32_t>(workspace, w.cnt);
+  m.idx = at<int32_t>(workspace, w.idx);
+  m.tcnt = at<int32_t>(workspace, w.tcnt);
+  m.tidx = at<int32_t>(workspace, w.tidx);
+  m.status = at<uint32_t>(workspace, w.status);
+  m.dense = desc->thr == 0.0f;
+  // mass threshold 1 - thr in the kernel's 2^-40 fixed point
+  m.target_fx = (unsigned long long)std::llround((1.0 - (double)desc->thr) * 1099511627776.0);
+  const bool sta = desc->sta_t > 0;
+  m.sta_t = sta ? desc->sta_t / 2 : -1;
+  m.sta_h = sta ? desc->sta_h / 2 : -1;
+  m.sta_w = sta ? desc->sta_w / 2 : -1;
+  m.scale = (float)(1.0 / std::sqrt((double)g.d));
+  return cuda_status(launch_mask(m, g, s));
+}
+
+sa_status sparse_attn_fwd(const sa_desc* desc, const void* q, const void* k, const void* v,
+                          const void* workspace, size_t ws_bytes, void* out, void* stream) {
+  sa_status st = validate(desc);
+  if (st != SA_OK) return st;
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || !aligned(q, 16) ||
+      !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
+    return SA_ERR_INVALID_ARG;
+  const Geometry g = make_geometry(*desc);
+  st = check_ws(g, workspace, ws_bytes);
+  if (st != SA_OK) return st;
+  const WsLayout w = make_ws_layout(g);
+  AttnArgs a;
+  std::memset(&a, 0, sizeof(a));
+  if (!encode_patch_map(&a.map_q, q, g.BH, g.T, g.Hh, g.Ww, g.d, g.P) ||
+      !encode_patch_map(&a.map_k, k, g.BH, g.T, g.Hh, g.Ww, g.d, g.P) ||
+      !encode_patch_map(&a.map_v, v, g.BH, g.T, g.Hh, g.Ww, g.d, g.P))
+    return SA_ERR_CUDA;
+  a.out = out;
+  a.tcnt = at<int32_t>(workspace, w.tcnt);
+  a.tidx = at<int32_t>(workspace, w.tidx);
+  a.status = const_cast<uint32_t*>(at<uint32_t>(workspace, w.status));
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)g.d));
+  a.out_fp32 = desc->out_fp32;
+  a.debug_flags = desc->debug_flags;
+  return cuda_status(launch_attn(a, g, static_cast<cudaStream_t>(stream)));
+}
+
+sa_status sparse_attn_permute(const sa_desc* desc, const void* x, void* y, int inverse,
+                              void* stream) {
+  const sa_status st = validate(desc);
+  if (st != SA_OK) return st;
+  if (x == nullptr || y == nullptr || !aligned(x, 16) || !aligned(y, 16) ||
+      (inverse != 0 && inverse != 1))
+    return SA_ERR_INVALID_ARG;
+  const Geometry g = make_geometry(*desc);
+  const size_t bytes = size_t(g.BH) * g.S * g.d * 2;
+  const uintptr_t xb = reinterpret_cast<uintptr_t>(x), yb = reinterpret_cast<uintptr_t>(y);
+  if (xb < yb + bytes && yb < xb + bytes) return SA_ERR_INVALID_ARG;  // overlap
+  return cuda_status(launch_permute(x, y, g, inverse, static_cast<cudaStream_t>(stream)));
+}
+
+sa_status sparse_attn_get_mask(const sa_desc* desc, const void* workspace, size_t ws_bytes,
+                               sa_mask_views* views) {
+  sa_status st = validate(desc);
+  if (st != SA_OK) return st;
+  if (views == nullptr) return SA_ERR_INVALID_ARG;
+  const Geometry g = make_geometry(*desc);
+  st = check_ws(g, workspace, ws_bytes);
+  if (st != SA_OK) return st;
+  const WsLayout w = make_ws_layout(g);
+  views->qbar = at<float>(workspace, w.qbar);
+  views->kbar = at<float>(workspace, w.kbar);
+  views->cnt = at<int32_t>(workspace, w.cnt);
+  views->idx = at<int32_t>(workspace, w.idx);
+  views->tile_cnt = at<int32_t>(workspace, w.tcnt);
+  views->tile_idx = at<int32_t>(workspace, w.tidx);
+  views->nb = g.nb;
+  views->ntile = g.ntile;
+  return SA_OK;
+}
+
+sa_status sparse_attn_tile_blocks(const sa_desc* desc, int tile, int* qa, int* qb) {
+  const sa_status st = validate(desc);
+  if (st != SA_OK) return st;
+  const Geometry g = make_geometry(*desc);
+  if (qa == nullptr || qb == nullptr || tile < 0 || tile >= g.ntile) return SA_ERR_INVALID_ARG;
+  tile_blocks(g, tile, *qa, *qb);
+  return SA_OK;
+}
+
+sa_status sparse_attn_check(const sa_desc* desc, const void* workspace, size_t ws_bytes,
+                            void* stream) {
+  sa_status st = validate(desc);
+  if (st != SA_OK) return st;
+  const Geometry g = make_geometry(*desc);
+  st = check_ws(g, workspace, ws_bytes);
+  if (st != SA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return SA_ERR_CUDA;
+  uint32_t word = 0;
+  const WsLayout w = make_ws_layout(g);
+  if (cudaMemcpy(&word, at<uint32_t>(workspace, w.status), sizeof(word), cudaMemcpyDeviceToHost) !=
+      cudaSuccess)
+    return SA_ERR_CUDA;
+  return word ? SA_ERR_DEVICE_TIMEOUT : SA_OK;
+}
+
+const char* sparse_attn_status_string(sa_status status) {
+  switch (status) {
+    case SA_OK: return "ok";
+    case SA_ERR_INVALID_ARG: return "invalid argument";
+    case SA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SA_ERR_WORKSPACE: return "workspace too small";
+    case SA_ERR_CUDA: return "CUDA runtime error";
+    case SA_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait ran out (device status set)";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

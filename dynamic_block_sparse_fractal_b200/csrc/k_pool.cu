@@ -1,0 +1,110 @@
+// Block pooling of Q and K ("Sottocampionamento", NABLA Metodologia 2):
+// Qbar[bh][b] = mean of the N = P*P tokens of block b, i.e. of the P x P
+// patch (hp, wp) of frame t, read straight from the natural layout (the
+// fractal flattening is only an addressing here).
+//
+// One warp per (bh, block) and tensor; each lane owns d/32 channels and
+// streams the 64 token rows with coalesced 8-byte (d = 128) or 4-byte loads,
+// accumulating in fp32. HBM-bound: reads Q and K once, writes Qbar, Kbar.
+#include <cuda_bf16.h>
+
+#include "kernels.cuh"
+
+namespace sa {
+
+template <int D>
+__global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ q,
+                                                   const __nv_bfloat16* __restrict__ k,
+                                                   float* __restrict__ qbar,
+                                                   float* __restrict__ kbar, Geometry g) {
+  constexpr int kPerLane = D / 32;  // 4 or 2 channels per lane
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long unit = long(blockIdx.x) * 8 + warp;  // (tensor, bh, b)
+  const long per_tensor = long(g.BH) * g.nb;
+  if (unit >= 2 * per_tensor) return;
+  const int which = int(unit / per_tensor);
+  const long rest = unit - which * per_tensor;
+  const int bh = int(rest / g.nb), b = int(rest - long(bh) * g.nb);
+  int t, hp, wp;
+  block_coords(g, b, t, hp, wp);
+  const __nv_bfloat16* src = (which == 0 ? q : k) + (size_t(bh) * g.S) * D + lane * kPerLane;
+  float acc[kPerLane];
+#pragma unroll
+  for (int i = 0; i < kPerLane; ++i) acc[i] = 0.f;
+  const size_t frame0 = size_t(t) * g.Hh * g.Ww;
+#pragma unroll 4
+  for (int hi = 0; hi < 8; ++hi) {
+    const size_t row0 = frame0 + size_t(hp * 8 + hi) * g.Ww + wp * 8;
+    float2 raw[8];
+#pragma unroll
+    for (int wi = 0; wi < 8; ++wi) {
+      const __nv_bfloat16* p = src + (row0 + wi) * D;
+      if constexpr (kPerLane == 4) {
+        raw[wi] = __ldg(reinterpret_cast<const float2*>(p));
+      } else {
+        raw[wi].x = __ldg(reinterpret_cast<const float*>(p));
+      }
+    }
+#pragma unroll
+    for (int wi = 0; wi < 8; ++wi) {
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[wi]);
+#pragma unroll
+      for (int i = 0; i < kPerLane / 2; ++i) {
+        const float2 f = __bfloat1622float2(h[i]);
+        acc[2 * i] += f.x;
+        acc[2 * i + 1] += f.y;
+      }
+    }
+  }
+  float* dst = (which == 0 ? qbar : kbar) + (size_t(bh) * g.nb + b) * D + lane * kPerLane;
+  const float inv = 1.0f / 64.0f;  // exact: N = 64
+#pragma unroll
+  for (int i = 0; i < kPerLane; ++i) dst[i] = acc[i] * inv;
+}
+
+cudaError_t launch_pool(const void* q, const void* k, float* qbar, float* kbar, const Geometry& g,
+                        cudaStream_t stream) {
+  const long units = 2L * g.BH * g.nb;
+  const unsigned grid = unsigned((units + 7) / 8);
+  const auto* qq = static_cast<const __nv_bfloat16*>(q);
+  const auto* kk = static_cast<const __nv_bfloat16*>(k);
+  if (g.d == 128)
+    pool_kernel<128><<<grid, 256, 0, stream>>>(qq, kk, qbar, kbar, g);
+  else
+    pool_kernel<64><<<grid, 256, 0, stream>>>(qq, kk, qbar, kbar, g);
+  return cudaGetLastError();
+}
+
+// Fractal flattening as an explicit copy: position p = b*64 + hi*8 + wi of a
+// head holds the natural token (t, hp*8 + hi, wp*8 + wi) of block b. One warp
+// per (bh, block, patch row hi): 8 tokens x d channels, 16-byte vectors.
+__global__ void __launch_bounds__(256) permute_kernel(const uint4* __restrict__ x,
+                                                      uint4* __restrict__ y, Geometry g,
+                                                      int inverse) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long unit = long(blockIdx.x) * 8 + warp;  // (bh, b, hi)
+  if (unit >= long(g.BH) * g.nb * 8) return;
+  const int hi = int(unit & 7);
+  const long bb = unit >> 3;
+  const int bh = int(bb / g.nb), b = int(bb - long(bh) * g.nb);
+  int t, hp, wp;
+  block_coords(g, b, t, hp, wp);
+  const int vec_per_row = g.d / 8;  // 16-byte vectors per token row
+  const size_t nat = size_t(t) * g.Hh * g.Ww + size_t(hp * 8 + hi) * g.Ww + wp * 8;
+  const size_t frac = size_t(b) * 64 + hi * 8;
+  const size_t head = size_t(bh) * g.S;
+  const size_t src0 = (head + (inverse ? frac : nat)) * vec_per_row;
+  const size_t dst0 = (head + (inverse ? nat : frac)) * vec_per_row;
+  // the 8 tokens of a patch row are contiguous in both orders
+  for (int i = lane; i < 8 * vec_per_row; i += 32) y[dst0 + i] = __ldg(x + src0 + i);
+}
+
+cudaError_t launch_permute(const void* x, void* y, const Geometry& g, int inverse,
+                           cudaStream_t stream) {
+  const long units = long(g.BH) * g.nb * 8;
+  permute_kernel<<<unsigned((units + 7) / 8), 256, 0, stream>>>(
+      static_cast<const uint4*>(x), static_cast<uint4*>(y), g, inverse);
+  return cudaGetLastError();
+}
+
+}  // namespace sa

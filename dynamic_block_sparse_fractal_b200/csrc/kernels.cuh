@@ -1,0 +1,50 @@
+// Launch wrappers of the library's kernels (host side). Each returns the
+// launch's cudaError_t; argument validation happens before any of them.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "layout.cuh"
+
+namespace sa {
+
+cudaError_t launch_pool(const void* q, const void* k, float* qbar, float* kbar, const Geometry& g,
+                        cudaStream_t stream);
+
+cudaError_t launch_permute(const void* x, void* y, const Geometry& g, int inverse,
+                           cudaStream_t stream);
+
+// Reduced map + CDF threshold + STA union -> per-q-block lists and per-tile
+// union lists. target_fx = round((1 - thr) * 2^40) (mass threshold in the
+// kernel's fixed point); dense = (thr == 0).
+struct MaskArgs {
+  const float* qbar;
+  const float* kbar;
+  int32_t* cnt;
+  int32_t* idx;
+  int32_t* tcnt;
+  int32_t* tidx;
+  uint32_t* status;
+  unsigned long long target_fx;
+  int dense;
+  int sta_t, sta_h, sta_w;  // half-widths (window / 2), -1 = no STA
+  float scale;              // 1 / sqrt(d)
+};
+cudaError_t launch_mask(const MaskArgs& a, const Geometry& g, cudaStream_t stream);
+size_t mask_smem_bytes(const Geometry& g);
+
+struct AttnArgs {
+  CUtensorMap map_q, map_k, map_v;  // 5-D patch maps, see tma_host.h
+  void* out;
+  const int32_t* tcnt;
+  const int32_t* tidx;
+  uint32_t* status;
+  float scale_log2;  // log2(e) / sqrt(d)
+  int out_fp32;
+  int debug_flags;
+};
+cudaError_t launch_attn(const AttnArgs& a, const Geometry& g, cudaStream_t stream);
+
+}  // namespace sa

@@ -1,0 +1,101 @@
+// Geometry shared by the host entry points and the kernels: block grid,
+// query-tile pairing and the workspace layout.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/sparse_attn.h"
+
+namespace sa {
+
+#define SA_HD __host__ __device__ __forceinline__
+
+struct Geometry {
+  int BH, T, Hh, Ww, d, P, N;
+  int nh, nw;   // patches per frame along h and w
+  int nb;       // blocks per head = T * nh * nw
+  int ntile;    // query tiles per head
+  int S;        // tokens per head
+};
+
+SA_HD Geometry make_geometry(const sa_desc& s) {
+  Geometry g;
+  g.BH = s.B * s.H;
+  g.T = s.T;
+  g.Hh = s.Hh;
+  g.Ww = s.Ww;
+  g.d = s.d;
+  g.P = s.P;
+  g.N = s.N;
+  g.nh = s.Hh / s.P;
+  g.nw = s.Ww / s.P;
+  g.nb = s.T * g.nh * g.nw;
+  g.S = s.T * s.Hh * s.Ww;
+  const int pairs_t = (s.T / 2) * g.nh * g.nw;
+  g.ntile = pairs_t + ((s.T & 1) ? g.nh * ((g.nw + 1) / 2) : 0);
+  return g;
+}
+
+// Block b (fractal block order) -> frame t, patch row hp, patch column wp.
+SA_HD void block_coords(const Geometry& g, int b, int& t, int& hp, int& wp) {
+  const int per_frame = g.nh * g.nw;
+  t = b / per_frame;
+  const int r = b - t * per_frame;
+  hp = r / g.nw;
+  wp = r - hp * g.nw;
+}
+
+// Query tile -> the two q-blocks it holds (qb = -1 when alone). Pairs are
+// the same patch in frames (2i, 2i+1); an odd last frame pairs neighbouring
+// patch columns.
+SA_HD void tile_blocks(const Geometry& g, int tile, int& qa, int& qb) {
+  const int per_frame = g.nh * g.nw;
+  const int pairs_t = (g.T / 2) * per_frame;
+  if (tile < pairs_t) {
+    const int tp = tile / per_frame;
+    qa = 2 * tp * per_frame + (tile - tp * per_frame);
+    qb = qa + per_frame;
+  } else {
+    const int i = tile - pairs_t;
+    const int half = (g.nw + 1) / 2;
+    const int hp = i / half, wq = i - hp * half;
+    qa = (g.T - 1) * per_frame + hp * g.nw + 2 * wq;
+    qb = (2 * wq + 1 < g.nw) ? qa + 1 : -1;
+  }
+}
+
+// Workspace: every region starts on a 256-byte boundary.
+struct WsLayout {
+  size_t status;   // uint32 device status word (+ padding)
+  size_t qbar;     // float [BH][nb][d]
+  size_t kbar;     // float [BH][nb][d]
+  size_t cnt;      // int32 [BH][nb]
+  size_t idx;      // int32 [BH][nb][nb]
+  size_t tcnt;     // int32 [BH][ntile]
+  size_t tidx;     // int32 [BH][ntile][nb]
+  size_t total;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline WsLayout make_ws_layout(const Geometry& g) {
+  WsLayout w;
+  size_t o = 0;
+  w.status = o; o = align256(o + 256);
+  w.qbar = o; o = align256(o + sizeof(float) * size_t(g.BH) * g.nb * g.d);
+  w.kbar = o; o = align256(o + sizeof(float) * size_t(g.BH) * g.nb * g.d);
+  w.cnt = o; o = align256(o + sizeof(int32_t) * size_t(g.BH) * g.nb);
+  w.idx = o; o = align256(o + sizeof(int32_t) * size_t(g.BH) * g.nb * g.nb);
+  w.tcnt = o; o = align256(o + sizeof(int32_t) * size_t(g.BH) * g.ntile);
+  w.tidx = o; o = align256(o + sizeof(int32_t) * size_t(g.BH) * g.ntile * g.nb);
+  w.total = o;
+  return w;
+}
+
+// Union-list entry: k-block id | keep bit of the tile's first q-block << 16
+// | keep bit of the second q-block << 17.
+constexpr int kEntryBlockMask = 0xFFFF;
+constexpr int kEntryKeepA = 1 << 16;
+constexpr int kEntryKeepB = 1 << 17;
+
+}  // namespace sa

@@ -1,0 +1,46 @@
+// Host-side construction of TMA tensor maps. The driver entry point is looked
+// up through the runtime, so the library needs no link against libcuda.
+#pragma once
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace sa {
+
+inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// bf16 tensor [BH][T][Hh][Ww][d] (natural video order, d innermost) seen as a
+// 5-D TMA tensor whose box is one 64-channel slice of a P x P spatial patch of
+// one frame: P*P token rows of 128 bytes, written to shared memory with the
+// 128-byte swizzle. Coordinates are (channel, w, h, t, bh).
+inline bool encode_patch_map(CUtensorMap* map, const void* base, int BH, int T, int Hh, int Ww,
+                             int d, int P) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[5] = {cuuint64_t(d), cuuint64_t(Ww), cuuint64_t(Hh), cuuint64_t(T),
+                        cuuint64_t(BH)};
+  cuuint64_t row = cuuint64_t(d) * 2;
+  cuuint64_t strides[4] = {row, row * Ww, row * Ww * Hh, row * Ww * Hh * T};
+  cuuint32_t box[5] = {64, cuuint32_t(P), cuuint32_t(P), 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace sa

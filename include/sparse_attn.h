@@ -1,0 +1,150 @@
+/*
+ * sparse_attn.h — C ABI of libsparse_attn.so: content-adaptive block-sparse
+ * self-attention over spatio-temporal video tokens, in the form of
+ * "NABLA - Neighborhood Adaptive Block-Level Attention per la Generazione
+ * Efficiente di Video" (gist.science/it/paper/2507.13546), section
+ * "Metodologia: NABLA".
+ *
+ * The path is split in two calls:
+ *   sparse_attn_plan  fractal flattening (as addressing) + block pooling of Q
+ *                     and K + reduced attention map + per-row CDF threshold
+ *                     + optional STA union  ->  block lists in a workspace;
+ *   sparse_attn_fwd   exact attention over the kept (q-block, k-block) pairs,
+ *                     written back in natural token order.
+ * One plan may serve many fwd calls with the same Q/K statistics.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     allocates nothing and keeps no state between calls.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream). Argument errors are reported before anything is launched.
+ *   - Q, K, V and the output use the natural video layout [B, H, S, d] with
+ *     S = T*Hh*Ww tokens ordered (t, h, w), t outermost, d innermost,
+ *     contiguous, bf16 (raw 16-bit storage), 16-byte aligned.
+ *   - Device-side failures (a bounded wait that ran out, an out-of-range block
+ *     index) are recorded in a status word inside the workspace and reported
+ *     by sparse_attn_check. No kernel of this library traps.
+ */
+#ifndef SPARSE_ATTN_H
+#define SPARSE_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Problem description. The method's parameters follow the NABLA page:
+ * P is the spatial patch edge of "Fractal Flattening" (Metodologia 1), N the
+ * block length of "Sottocampionamento" and the N x N attention-map block
+ * (Metodologia 2), thr the "CDF Thresholding" parameter (Metodologia 2), and
+ * (sta_t, sta_h, sta_w) the static window of "Integrazione Ibrida con STA"
+ * (Metodologia 3), in block units. */
+typedef struct sa_desc {
+  int B, H;          /* batch, heads */
+  int T, Hh, Ww;     /* latent grid: frames, height, width (S = T*Hh*Ww) */
+  int d;             /* head dimension: 64 or 128 */
+  int N, P;          /* block tokens and patch edge; requires N == P*P = 64,
+                        Hh % P == 0 and Ww % P == 0 */
+  float thr;         /* [0, 1): keep the smallest descending-probability set
+                        of k-blocks whose mass reaches 1 - thr; 0 = dense */
+  int sta_t, sta_h, sta_w; /* odd STA window in blocks, or 0,0,0 = no STA */
+  int out_fp32;      /* 0: output bf16; 1: output fp32 (same layout) */
+  int debug_flags;   /* 0 in normal use; SA_DEBUG_* bits for tests */
+} sa_desc;
+
+/* Test-only: the attention kernel's loader never signals its first K/V
+ * stage, so the compute warps' bounded wait runs out and the call reports
+ * SA_ERR_DEVICE_TIMEOUT from sparse_attn_check (no fault, no hang). */
+#define SA_DEBUG_STALL_LOADER 1
+
+typedef enum sa_status {
+  SA_OK = 0,
+  SA_ERR_INVALID_ARG = 1,     /* NULL pointer, non-positive size, thr out of
+                                 range, even STA window, misaligned pointer */
+  SA_ERR_UNSUPPORTED = 2,     /* valid but not implemented: d not in {64,128},
+                                 N != P*P, N != 64, grid not divisible by P */
+  SA_ERR_WORKSPACE = 3,       /* workspace smaller than
+                                 sparse_attn_workspace_size() */
+  SA_ERR_CUDA = 4,            /* a CUDA runtime call or launch failed */
+  SA_ERR_DEVICE_TIMEOUT = 5   /* a kernel's bounded wait ran out */
+} sa_status;
+
+/* Bytes of device workspace a plan for `desc` needs (written to *bytes). */
+sa_status sparse_attn_workspace_size(const sa_desc* desc, size_t* bytes);
+
+/* Builds the block mask M = M_nabla OR M_STA for every (batch, head):
+ *   1. fractal flattening: block b of a head is the P x P patch (hp, wp) of
+ *      frame t, b = (t*(Hh/P) + hp)*(Ww/P) + wp, tokens row-major inside it
+ *      (NABLA, Metodologia 1);
+ *   2. Qbar, Kbar = mean of the N tokens of each block, fp32 (Metodologia 2,
+ *      "Sottocampionamento");
+ *   3. A = row softmax(Qbar Kbar^T / sqrt(d)) (Metodologia 2, "Attenzione
+ *      Ridotta"), never materialised;
+ *   4. per row, k-block j is kept iff the mass of the blocks ranked before it
+ *      (descending probability, ties by ascending index) is below 1 - thr
+ *      (Metodologia 2, "CDF Thresholding"); thr == 0 keeps every block;
+ *   5. union with the STA window |dt|<=sta_t/2, |dhp|<=sta_h/2, |dwp|<=sta_w/2
+ *      (Metodologia 3).
+ * q, k: [B,H,S,d] bf16 device tensors in natural order. workspace: device
+ * buffer of at least sparse_attn_workspace_size() bytes, 256-byte aligned;
+ * its previous contents are ignored and overwritten. */
+sa_status sparse_attn_plan(const sa_desc* desc, const void* q, const void* k,
+                           void* workspace, size_t ws_bytes, void* stream);
+
+/* O_i = sum over kept k-blocks of softmax(q_i . k_j / sqrt(d)) v_j for every
+ * query token i, i.e. exact attention with every dropped N x N block at -inf
+ * ("Espansione", NABLA Metodologia 2), written to `out` [B,H,S,d] in natural
+ * token order (bf16, or fp32 if desc->out_fp32). q, k, v as for the plan; the
+ * workspace must hold a plan made for the same desc (q, k may differ from the
+ * plan's, e.g. when a plan is reused across steps). */
+sa_status sparse_attn_fwd(const sa_desc* desc, const void* q, const void* k,
+                          const void* v, const void* workspace, size_t ws_bytes,
+                          void* out, void* stream);
+
+/* Fractal flattening of one [B,H,S,d] bf16 tensor (inverse = 0: natural ->
+ * fractal order, position p of a head holds token perm[p]) or its inverse
+ * (inverse = 1). x and y must not overlap. The attention path itself reads
+ * the natural layout through TMA addressing and does not call this. */
+sa_status sparse_attn_permute(const sa_desc* desc, const void* x, void* y,
+                              int inverse, void* stream);
+
+/* Device views into a planned workspace (pointers into `workspace`; valid as
+ * long as it is). Block indices are in fractal block order. */
+typedef struct sa_mask_views {
+  const float* qbar;     /* [B*H][nb][d] pooled queries */
+  const float* kbar;     /* [B*H][nb][d] pooled keys */
+  const int32_t* cnt;    /* [B*H][nb] kept k-blocks per q-block */
+  const int32_t* idx;    /* [B*H][nb][nb] kept k-block ids, ascending, first
+                            cnt entries valid */
+  const int32_t* tile_cnt;  /* [B*H][ntile] union length per query tile */
+  const int32_t* tile_idx;  /* [B*H][ntile][nb] union entries: k-block id in
+                               bits 0-15, bit 16 = first q-block keeps it,
+                               bit 17 = second q-block keeps it */
+  int nb;                /* blocks per head */
+  int ntile;             /* query tiles per head (pairs of q-blocks) */
+} sa_mask_views;
+
+sa_status sparse_attn_get_mask(const sa_desc* desc, const void* workspace,
+                               size_t ws_bytes, sa_mask_views* views);
+
+/* Query tile -> its two q-blocks (second = -1 for a lone block). Tiles pair
+ * block (t, hp, wp) with (t+1, hp, wp) for even t; with an odd T the last
+ * frame pairs (hp, wp) with (hp, wp+1). */
+sa_status sparse_attn_tile_blocks(const sa_desc* desc, int tile, int* qa, int* qb);
+
+/* Waits for `stream`, then reports SA_ERR_DEVICE_TIMEOUT if a kernel of the
+ * last plan/fwd on this workspace recorded a device-side failure, SA_ERR_CUDA
+ * if the stream holds a CUDA error, else SA_OK. */
+sa_status sparse_attn_check(const sa_desc* desc, const void* workspace,
+                            size_t ws_bytes, void* stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char* sparse_attn_status_string(sa_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSE_ATTN_H */

@@ -1,0 +1,97 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+the header declares, and rejects bad arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from dynamic_block_sparse_fractal_b200 import api, workloads as W
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                      "include", "sparse_attn.h")
+FAKE = ctypes.c_void_p(0x10000000)  # never dereferenced: validation fails first
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"\b(sparse_attn_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = api.lib()
+    names = declared_functions()
+    assert set(names) == set(api.SYMBOLS)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_workspace_size_and_validation():
+    d = api.desc_for(W.HUNYUAN)
+    assert api.workspace_size(d) > 0
+    bad = [
+        dict(d=96), dict(P=4, N=16), dict(Hh=44), dict(thr=1.0), dict(thr=-0.1),
+        dict(thr=float("nan")), dict(sta=(2, 3, 3)), dict(sta=(3, 0, 3)), dict(B=0),
+    ]
+    expect = [api.SA_ERR_UNSUPPORTED, api.SA_ERR_UNSUPPORTED, api.SA_ERR_UNSUPPORTED,
+              api.SA_ERR_INVALID_ARG, api.SA_ERR_INVALID_ARG, api.SA_ERR_INVALID_ARG,
+              api.SA_ERR_INVALID_ARG, api.SA_ERR_INVALID_ARG, api.SA_ERR_INVALID_ARG]
+    base = dict(B=1, H=2, T=4, Hh=16, Ww=16, d=128, thr=0.1, sta=(0, 0, 0), N=64, P=8)
+    for b, e in zip(bad, expect):
+        kw = dict(base, **b)
+        n = ctypes.c_size_t()
+        st = api.lib().sparse_attn_workspace_size(ctypes.byref(api.make_desc(**kw)),
+                                                  ctypes.byref(n))
+        assert st == e, (b, st)
+    # too many blocks per head for the mask kernel's shared memory
+    big = api.make_desc(1, 1, 100, 64, 64, 128, 0.1)
+    n = ctypes.c_size_t()
+    assert api.lib().sparse_attn_workspace_size(ctypes.byref(big), ctypes.byref(n)) == \
+        api.SA_ERR_UNSUPPORTED
+
+
+def test_entry_points_reject_before_launch():
+    L = api.lib()
+    d = api.desc_for(W.TINY)
+    need = api.workspace_size(d)
+    st = L.sparse_attn_plan(ctypes.byref(d), FAKE, FAKE, FAKE, need - 1, None)
+    assert st == api.SA_ERR_WORKSPACE
+    st = L.sparse_attn_plan(ctypes.byref(d), None, FAKE, FAKE, need, None)
+    assert st == api.SA_ERR_INVALID_ARG
+    st = L.sparse_attn_plan(ctypes.byref(d), ctypes.c_void_p(0x10000008), FAKE, FAKE, need, None)
+    assert st == api.SA_ERR_INVALID_ARG  # q not 16-byte aligned
+    st = L.sparse_attn_fwd(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, need - 256, FAKE, None)
+    assert st == api.SA_ERR_WORKSPACE
+    st = L.sparse_attn_fwd(ctypes.byref(d), FAKE, FAKE, FAKE, ctypes.c_void_p(0x10000010),
+                           need, FAKE, None)
+    assert st == api.SA_ERR_INVALID_ARG  # workspace not 256-byte aligned
+    st = L.sparse_attn_permute(ctypes.byref(d), FAKE, FAKE, 0, None)
+    assert st == api.SA_ERR_INVALID_ARG  # x and y overlap
+    st = L.sparse_attn_permute(ctypes.byref(d), FAKE, FAKE, 2, None)
+    assert st == api.SA_ERR_INVALID_ARG
+    v = api.SaMaskViews()
+    assert L.sparse_attn_get_mask(ctypes.byref(d), FAKE, need - 1, ctypes.byref(v)) == \
+        api.SA_ERR_WORKSPACE
+    assert L.sparse_attn_check(ctypes.byref(d), FAKE, 0, None) == api.SA_ERR_WORKSPACE
+    assert L.sparse_attn_get_mask(None, FAKE, need, ctypes.byref(v)) == api.SA_ERR_INVALID_ARG
+    assert api.status_string(api.SA_ERR_DEVICE_TIMEOUT).startswith("a kernel")
+
+
+@pytest.mark.parametrize("T,Hh,Ww", [(4, 8, 8), (33, 48, 80), (21, 32, 56), (3, 8, 24), (1, 16, 8)])
+def test_tile_pairing_covers_every_block_once(T, Hh, Ww):
+    d = api.make_desc(1, 1, T, Hh, Ww, 128, 0.1)
+    nh, nw = Hh // 8, Ww // 8
+    nb = T * nh * nw
+    seen = []
+    ntile = (T // 2) * nh * nw + (T % 2) * nh * ((nw + 1) // 2)
+    for i in range(ntile):
+        qa, qb = api.tile_blocks(d, i)
+        seen.append(qa)
+        if qb >= 0:
+            seen.append(qb)
+            ta, tb = qa // (nh * nw), qb // (nh * nw)
+            # same patch in consecutive frames, or neighbours in the last odd frame
+            assert (tb == ta + 1 and qb - qa == nh * nw) or (ta == tb == T - 1 and qb == qa + 1)
+    assert sorted(seen) == list(range(nb))
+    with pytest.raises(api.SparseAttnError):
+        api.tile_blocks(d, ntile)

@@ -1,0 +1,249 @@
+"""CUDA path (through the C ABI) vs the fp64 CPU oracle, on the seeded
+workloads and on edge shapes. Masks: exact outside the ambiguity band
+(tests/parity.py); outputs: max-abs <= 2e-2, mean-abs <= 2e-3."""
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from dynamic_block_sparse_fractal_b200 import api, workloads as W
+from tests import parity
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+
+@functools.lru_cache(maxsize=2)
+def host_inputs(w):
+    q, k, v = W.make_inputs(w)
+    return (q.reshape(w.BH, w.S, w.d), k.reshape(w.BH, w.S, w.d), v.reshape(w.BH, w.S, w.d))
+
+
+def to_dev(bits, w):
+    t = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+    return t.reshape(w.B, w.H, w.S, w.d).cuda()
+
+
+def run(w, out_fp32=False, debug_flags=0, inputs=None):
+    """plan + fwd on the GPU; returns (out [BH,S,d] float np, gpu mask, views)."""
+    q, k, v = inputs if inputs is not None else host_inputs(w)
+    qd, kd, vd = to_dev(q, w), to_dev(k, w), to_dev(v, w)
+    desc = api.desc_for(w, out_fp32=out_fp32, debug_flags=debug_flags)
+    ws = api.alloc_workspace(desc)
+    api.plan(desc, qd, kd, ws)
+    out = torch.empty(qd.shape, device="cuda",
+                      dtype=torch.float32 if out_fp32 else torch.bfloat16)
+    api.fwd(desc, qd, kd, vd, ws, out)
+    st = api.check(desc, ws)
+    assert st == api.SA_OK, api.status_string(st)
+    views = api.get_mask(desc, ws)
+    cnt = views["cnt"].cpu().numpy()
+    idx = views["idx"].cpu().numpy()
+    gm = parity.lists_to_mask(cnt, idx)
+    return out.float().cpu().numpy().reshape(w.BH, w.S, w.d), gm, views, desc, ws
+
+
+def oracle_mask(w, heads=None):
+    q, k, _ = host_inputs(w)
+    sel = range(w.BH) if heads is None else heads
+    return oracle.nabla_mask(q[list(sel)], k[list(sel)], w.T, w.Hh, w.Ww, w.P, w.N, w.thr, w.sta)
+
+
+def check_mask(w, gm, heads=None):
+    M, Mn, A = oracle_mask(w, heads)
+    sel = list(range(w.BH) if heads is None else heads)
+    r = parity.compare_masks(gm[sel], M, Mn, A, w.thr)
+    assert r["bad"] == 0, r
+    assert r["sta_missing"] == 0, r
+    assert r["min_mass_margin"] >= -parity.MASK_BAND, r
+    return r
+
+
+def check_out_full(w, out, gm, bf16_out=True):
+    q, k, v = host_inputs(w)
+    ref, _ = oracle.nabla_attention(q, k, v, w.T, w.Hh, w.Ww, w.P, w.N, w.thr, w.sta, mask=gm)
+    r = parity.out_check(out, ref, bf16_out)
+    assert r["ok"], r
+    return r
+
+
+def check_out_sampled(w, out, gm, heads, n_tok=96, seed=0, bf16_out=True):
+    q, k, v = host_inputs(w)
+    rng = np.random.default_rng(seed)
+    got, refs = [], []
+    for bh in heads:
+        toks = rng.choice(w.S, size=n_tok, replace=False)
+        refs.append(oracle.attention_head(q[bh], k[bh], v[bh], w.T, w.Hh, w.Ww, w.P, w.N, gm[bh],
+                                          tokens=toks))
+        got.append(out[bh][toks])
+    r = parity.out_check(np.concatenate(got), np.concatenate(refs), bf16_out)
+    assert r["ok"], r
+    return r
+
+
+# ---------------------------------------------------------------- small, in full
+
+@pytest.mark.parametrize("out_fp32", [False, True])
+def test_tiny_full(out_fp32):
+    w = W.TINY
+    out, gm, *_ = run(w, out_fp32=out_fp32)
+    check_mask(w, gm)
+    check_out_full(w, out, gm, bf16_out=not out_fp32)
+
+
+@pytest.mark.parametrize("out_fp32", [False, True])
+def test_8k_full(out_fp32):
+    w = W.W8K
+    out, gm, *_ = run(w, out_fp32=out_fp32)
+    check_mask(w, gm)
+    check_out_full(w, out, gm, bf16_out=not out_fp32)
+
+
+def test_permute_bit_exact():
+    w = W.W8K
+    q, _, _ = host_inputs(w)
+    x = to_dev(q, w)
+    desc = api.desc_for(w)
+    y = torch.empty_like(x)
+    api.permute(desc, x, y)
+    perm = oracle.fractal_order(w.T, w.Hh, w.Ww, w.P)
+    got = y.view(torch.int16).cpu().numpy().reshape(w.BH, w.S, w.d).view(np.uint16)
+    assert np.array_equal(got, oracle.flatten(q, perm))
+    z = torch.empty_like(x)
+    api.permute(desc, y, z, inverse=True)
+    assert torch.equal(z.view(torch.int16), x.view(torch.int16))
+
+
+def test_pooled_blocks_match_oracle():
+    w = W.W8K
+    _, _, views, *_ = run(w)
+    q, k, _ = host_inputs(w)
+    for bh in (0, 5, w.BH - 1):
+        for name, x in (("qbar", q), ("kbar", k)):
+            ref = oracle.pooled_head(x[bh], w.T, w.Hh, w.Ww, w.P, w.N)
+            got = views[name][bh].cpu().numpy().astype(np.float64)
+            assert np.abs(got - ref).max() <= 1e-6 * max(1.0, np.abs(ref).max())
+
+
+def test_union_lists_match_per_block_lists():
+    w = W.W8K
+    _, gm, views, desc, _ = run(w)
+    tc = views["tile_cnt"].cpu().numpy()
+    ti = views["tile_idx"].cpu().numpy()
+    for bh in range(w.BH):
+        for t in range(views["ntile"]):
+            qa, qb = api.tile_blocks(desc, t)
+            ma = gm[bh, qa]
+            mb = gm[bh, qb] if qb >= 0 else np.zeros_like(ma)
+            ent = ti[bh, t, :tc[bh, t]]
+            blocks = ent & 0xFFFF
+            assert np.array_equal(blocks, np.nonzero(ma | mb)[0])
+            assert np.array_equal((ent >> 16) & 1, ma[blocks].astype(np.int32))
+            assert np.array_equal((ent >> 17) & 1, mb[blocks].astype(np.int32))
+
+
+# ---------------------------------------------------------------- edge shapes
+
+EDGE = [
+    # ragged: nb = 30 (not a multiple of the 16-row mask tile or 64-block chunk),
+    # odd T with odd patch columns -> lone q-blocks; batch > 1
+    W.Workload("edge_ragged", B=2, H=3, d=128, T=5, Hh=16, Ww=24, thr=0.15, seed=7,
+               v_positional=True),
+    W.Workload("edge_d64_sta", B=1, H=2, d=64, T=3, Hh=24, Ww=16, thr=0.2, sta=(1, 3, 1),
+               seed=8, v_positional=True),
+    W.Workload("edge_thr_high", B=1, H=2, d=128, T=4, Hh=16, Ww=16, thr=0.99, seed=9),
+    W.Workload("edge_sta_covers_grid", B=1, H=2, d=128, T=2, Hh=16, Ww=16, thr=0.5,
+               sta=(5, 5, 5), seed=10),
+    W.Workload("edge_single_block", B=1, H=1, d=128, T=1, Hh=8, Ww=8, thr=0.1, seed=11),
+    W.Workload("edge_flat_noise", B=1, H=2, d=128, T=4, Hh=16, Ww=32, thr=0.1, scale=0.0,
+               seed=12),
+]
+
+
+@pytest.mark.parametrize("w", EDGE, ids=[e.name for e in EDGE])
+def test_edge_shapes(w):
+    out, gm, *_ = run(w)
+    check_mask(w, gm)
+    check_out_full(w, out, gm)
+
+
+def test_dense_threshold_matches_sdpa():
+    w = W.W8K.with_(thr=0.0, sta=(0, 0, 0))
+    out, gm, *_ = run(w, out_fp32=True)
+    assert gm.all()
+    q, k, v = (to_dev(x, w) for x in host_inputs(w))
+    # fp32 SDPA on the same bf16 values (torch's own kernel, as a second anchor)
+    ref = torch.nn.functional.scaled_dot_product_attention(q.float(), k.float(), v.float())
+    r = parity.out_check(out, ref.cpu().numpy().reshape(w.BH, w.S, w.d).astype(np.float64), False)
+    assert r["ok"], r
+    check_out_sampled(w, out, gm, heads=(0, 7), bf16_out=False)
+
+
+def test_deterministic_and_plan_reuse():
+    w = W.W8K
+    q, k, v = (to_dev(x, w) for x in host_inputs(w))
+    desc = api.desc_for(w)
+    ws1, ws2 = api.alloc_workspace(desc), api.alloc_workspace(desc)
+    api.plan(desc, q, k, ws1)
+    api.plan(desc, q, k, ws2)
+    m1, m2 = api.get_mask(desc, ws1), api.get_mask(desc, ws2)
+    for key in ("cnt", "tile_cnt"):
+        assert torch.equal(m1[key], m2[key])
+    o1, o2 = torch.empty_like(q), torch.empty_like(q)
+    api.fwd(desc, q, k, v, ws1, o1)
+    api.fwd(desc, q, k, v, ws1, o2)  # one plan, two forwards
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+    assert api.check(desc, ws1) == api.SA_OK
+
+
+def test_device_timeout_is_reported_and_context_survives():
+    w = W.TINY
+    q, k, v = (to_dev(x, w) for x in host_inputs(w))
+    desc = api.desc_for(w, debug_flags=api.SA_DEBUG_STALL_LOADER)
+    ws = api.alloc_workspace(desc)
+    api.plan(desc, q, k, ws)
+    out = torch.zeros_like(q)
+    api.fwd(desc, q, k, v, ws, out)
+    assert api.check(desc, ws) == api.SA_ERR_DEVICE_TIMEOUT
+    # the context is still usable: a normal call afterwards succeeds
+    out2, gm, *_ = run(w)
+    check_out_full(w, out2, gm)
+
+
+# ---------------------------------------------------------------- full sizes
+
+def test_wan_full_size():
+    w = W.WAN
+    out, gm, *_ = run(w)
+    check_mask(w, gm)
+    check_out_sampled(w, out, gm, heads=(0, 6, 11))
+
+
+def test_hunyuan_full_size():
+    w = W.HUNYUAN
+    out, gm, *_ = run(w)
+    r = check_mask(w, gm)
+    assert r["density"] < 0.2, r
+    check_out_sampled(w, out, gm, heads=(0, 13, 23), n_tok=64)
+
+
+SWEEP_FULL = [0, 7, 14, 21, 28, 35, 47]  # spans thr, STA on/off and every scale
+
+
+@pytest.mark.parametrize("k", SWEEP_FULL)
+def test_sweep_full_size(k):
+    w = W.sweep(k)
+    out, gm, *_ = run(w)
+    check_mask(w, gm, heads=(0, 11, 23))
+    check_out_sampled(w, out, gm, heads=(0, 23), n_tok=48)
+
+
+@pytest.mark.parametrize("k", range(W.N_SWEEP))
+def test_sweep_all_variants_small_grid(k):
+    # every (thr, STA, scale) combination on a 2-frame crop of the sweep grid
+    w = W.sweep(k).with_(H=2, T=2)
+    out, gm, *_ = run(w)
+    check_mask(w, gm)
+    check_out_full(w, out, gm)
