@@ -104,7 +104,9 @@ sa_status sparse_attn_plan(const sa_desc* desc, const void* q, const void* k, vo
   m.sta_h = sta ? desc->sta_h / 2 : -1;
   m.sta_w = sta ? desc->sta_w / 2 : -1;
   m.scale = (float)(1.0 / std::sqrt((double)g.d));
-  return cuda_status(launch_mask(m, g, s));
+  e = launch_mask(m, g, s);
+  if (e != cudaSuccess) return SA_ERR_CUDA;
+  return cuda_status(launch_tile_order(m.tcnt, at<int32_t>(workspace, w.order), g, s));
 }
 
 sa_status sparse_attn_fwd(const sa_desc* desc, const void* q, const void* k, const void* v,
@@ -127,6 +129,7 @@ sa_status sparse_attn_fwd(const sa_desc* desc, const void* q, const void* k, con
   a.out = out;
   a.tcnt = at<int32_t>(workspace, w.tcnt);
   a.tidx = at<int32_t>(workspace, w.tidx);
+  a.order = at<int32_t>(workspace, w.order);
   a.status = const_cast<uint32_t*>(at<uint32_t>(workspace, w.status));
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)g.d));
   a.out_fp32 = desc->out_fp32;

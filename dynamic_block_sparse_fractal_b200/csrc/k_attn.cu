@@ -2,25 +2,36 @@
 // ("Espansione", NABLA Metodologia 2: every dropped N x N block is -inf), on
 // the sm_100a tensor cores.
 //
-// A CTA computes one query tile of 128 rows = two q-blocks (64 rows each) of
-// one head, iterating over the union of their kept k-block lists two
-// k-blocks (128 keys) per step. Rows of a q-block that does not keep a
-// k-block see it as -inf (no exponentials are evaluated for it).
+// A query tile is 128 rows = two q-blocks (64 rows each) of one head; it runs
+// over the union of the two blocks' kept k-block lists, two k-blocks (128
+// keys) per step. Rows of a q-block that does not keep a k-block see it as
+// -inf and evaluate no exponentials for it.
 //
-//   warp 0      TMA producer: Q tile once, then K/V of each step into a
-//               2-stage ring. Q/K/V are read in natural layout through 5-D
-//               tensor maps whose box is one 8x8 patch of one frame, so the
-//               fractal flattening is pure addressing.
-//   warp 1      owns TMEM (512 columns) and issues tcgen05.mma:
-//                 S_j  = Q K_j^T  (SS, M=128, N=64*nblk, K=d) -> TMEM S[j%2]
-//                 O   += P_j V_j  (TS: P from TMEM, V MN-major from smem)
-//               S_{j+1} is issued before PV_j so the tensor core works while
-//               the softmax warps process S_j.
-//   warps 2-5   one thread per query row (TMEM lane): online softmax in fp32
-//               (exp2 domain), P written back as bf16 over S in TMEM, O
-//               rescaled in TMEM only when the running max grows by more than
-//               2^8 (exact after the final 1/l), epilogue stores O / l to the
-//               row's natural token position.
+// A CTA holds two tiles, A and B (consecutive entries of the head's
+// heaviest-first tile order), so that the tensor core works on one tile while
+// the softmax warps of the other run:
+//
+//   warp 0      TMA producer: the two Q tiles, then one 32 KB ring slot per
+//               MMA (a K pair for S, a V pair for PV) in exactly the order the
+//               MMA warp consumes them. Q/K/V are read in natural layout
+//               through 5-D tensor maps whose box is one 8x8 patch of one
+//               frame, so the fractal flattening is pure addressing.
+//   warp 1      owns TMEM (S_A, S_B, O_A, O_B: 4 x 128 columns) and issues
+//               tcgen05.mma in the order
+//                 S_A0 S_B0 | PV_A0 S_A1 PV_B0 S_B1 | PV_A1 S_A2 PV_B1 S_B2 | ...
+//               S_X = Q_X K^T (SS, M=128, N=64*nblk, K=d) -> TMEM S_X;
+//               O_X += P_X V (TS: P from TMEM over S_X, V MN-major in smem).
+//   warps 4-7   softmax of tile A, warps 8-11 softmax of tile B: one thread
+//               per query row (TMEM lane), online softmax in fp32 in the exp2
+//               domain, P written back as bf16 over S in TMEM, O rescaled in
+//               TMEM only when the running max grows by more than 2^8 (exact
+//               after the final 1/l), epilogue O / l -> natural token position.
+//   warps 2-3   idle.
+//
+// Ordering facts the pipeline relies on: tcgen05.mma ops issued by one thread
+// execute in order, and a tcgen05.commit tracks every op issued before it. So
+// when the softmax of tile X sees S_X(j) complete, PV_X(j-1) (issued before
+// S_X(j)) is complete too, and O_X may be rescaled without another wait.
 //
 // All waits are bounded (sm100.cuh); a wait that runs out records a status
 // bit, raises a CTA-wide abort flag, drains its own in-flight work and lets
@@ -28,6 +39,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "exp2_poly.cuh"
 #include "kernels.cuh"
 #include "sm100.cuh"
 
@@ -35,27 +47,75 @@ namespace sa {
 
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 384;
+constexpr int kSlots = 4;
 constexpr int kChunkBytes = 128 * 128;  // 128 rows x 128 B (64 bf16 channels)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int kMaxList = 2880;             // largest union: nb <= 2880 blocks
+
+__host__ __device__ constexpr uint32_t col_s(int x) { return uint32_t(x) * 128u; }
+__host__ __device__ constexpr uint32_t col_o(int x) { return 256u + uint32_t(x) * 128u; }
 
 template <int D>
 struct __align__(1024) AttnSmem {
-  uint8_t q[D / 64][kChunkBytes];
-  uint8_t k[2][D / 64][kChunkBytes];
-  uint8_t v[2][D / 64][kChunkBytes];
-  uint64_t q_full;
-  uint64_t kv_full[2];
-  uint64_t kv_empty[2];
+  uint8_t q[2][D / 64][kChunkBytes];
+  uint8_t slot[kSlots][D / 64][kChunkBytes];
+  int32_t list[2][kMaxList];  // the two tiles' union lists, staged once
+  uint64_t q_full[2];
+  uint64_t full[kSlots];
+  uint64_t empty[kSlots];
   uint64_t s_full[2];
   uint64_t p_full[2];
-  uint64_t pv_done;
-  uint64_t o_final;
+  uint64_t o_final[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
+};
+
+struct Tile {
+  int qa, qb;           // q-blocks (qb = -1: lone block)
+  int n_u;              // union length
+  int nsteps;           // ceil(n_u / 2)
+  const int32_t* list;  // union entries (shared-memory copy)
+};
+
+// The MMA issue order shared by the loader and the MMA warp.
+struct OpIter {
+  int n[2];
+  int j, sub;
+  __device__ OpIter(int na, int nb_) : j(0), sub(-2) {
+    n[0] = na;
+    n[1] = nb_;
+  }
+  // kind: 0 = S (consumes a K pair), 1 = PV (consumes a V pair)
+  __device__ bool next(int& kind, int& x, int& step) {
+    while (true) {
+      if (sub == -2) {
+        sub = -1;
+        if (n[0] > 0) { kind = 0; x = 0; step = 0; return true; }
+        continue;
+      }
+      if (sub == -1) {
+        sub = 0;
+        if (n[1] > 0) { kind = 0; x = 1; step = 0; return true; }
+        continue;
+      }
+      if (j >= (n[0] > n[1] ? n[0] : n[1])) return false;
+      const int s = sub, jj = j;
+      if (++sub == 4) {
+        sub = 0;
+        ++j;
+      }
+      const int t = s >> 1;
+      const int nt = t ? n[1] : n[0];
+      if ((s & 1) == 0) {
+        if (jj < nt) { kind = 1; x = t; step = jj; return true; }
+      } else {
+        if (jj + 1 < nt) { kind = 0; x = t; step = jj + 1; return true; }
+      }
+    }
+  }
 };
 
 __device__ __forceinline__ void fail(uint32_t* status, int* abort, uint32_t bit) {
@@ -63,37 +123,54 @@ __device__ __forceinline__ void fail(uint32_t* status, int* abort, uint32_t bit)
   *reinterpret_cast<volatile int*>(abort) = 1;
 }
 
+__device__ __forceinline__ int step_blocks(const Tile& t, int step) {
+  return (t.n_u - 2 * step) >= 2 ? 2 : 1;
+}
+
 }  // namespace
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ AttnArgs a, const Geometry g) {
-  const CUtensorMap* map_q = &a.map_q;
-  const CUtensorMap* map_k = &a.map_k;
-  const CUtensorMap* map_v = &a.map_v;
   extern __shared__ uint8_t smem_raw[];
   AttnSmem<D>& sm = *reinterpret_cast<AttnSmem<D>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile = blockIdx.x, bh = blockIdx.y;
-  int qa, qb;
-  tile_blocks(g, tile, qa, qb);
-  const int n_u = a.tcnt[size_t(bh) * g.ntile + tile];
-  const int32_t* list = a.tidx + (size_t(bh) * g.ntile + tile) * g.nb;
-  const int nsteps = (n_u + 1) >> 1;
+  const int bh = blockIdx.y;
+  const int pair = blockIdx.x;
+
+  Tile tile[2];
+#pragma unroll
+  for (int x = 0; x < 2; ++x) {
+    const int pos = 2 * pair + x;  // position in the head's tile order
+    tile[x].qa = tile[x].qb = -1;
+    tile[x].n_u = tile[x].nsteps = 0;
+    tile[x].list = nullptr;
+    if (pos < g.ntile) {
+      const int t = a.order[size_t(bh) * g.ntile + pos];
+      tile_blocks(g, t, tile[x].qa, tile[x].qb);
+      tile[x].n_u = a.tcnt[size_t(bh) * g.ntile + t];
+      tile[x].nsteps = (tile[x].n_u + 1) >> 1;
+      const int32_t* src = a.tidx + (size_t(bh) * g.ntile + t) * g.nb;
+      // every warp reads the lists at each step: stage them in shared memory
+      for (int i = threadIdx.x; i < tile[x].n_u; i += kThreads) sm.list[x][i] = src[i];
+    }
+    tile[x].list = sm.list[x];
+  }
   volatile int* abort = &sm.abort;
 
   if (threadIdx.x == 0) {
     sm.abort = 0;
-    mbar_init(&sm.q_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&sm.kv_full[s], 1);
-      mbar_init(&sm.kv_empty[s], 1);
-      mbar_init(&sm.s_full[s], 1);
-      mbar_init(&sm.p_full[s], 128);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&sm.q_full[x], 1);
+      mbar_init(&sm.s_full[x], 1);
+      mbar_init(&sm.p_full[x], 128);
+      mbar_init(&sm.o_final[x], 1);
     }
-    mbar_init(&sm.pv_done, 1);
-    mbar_init(&sm.o_final, 1);
+    for (int s = 0; s < kSlots; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1);
+    }
     mbar_init(&sm.drain, 1);
     fence_barrier_init();
   }
@@ -106,214 +183,255 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = sm.tmem_base;
 
-  if (nsteps > 0) {
-    if (warp == 0) {
-      // ------------------------------------------------------------ producer
-      if (lane == 0) {
-        prefetch_tensormap(map_q);
-        prefetch_tensormap(map_k);
-        prefetch_tensormap(map_v);
-        mbar_arrive_expect_tx(&sm.q_full, 128u * D * 2u);
+  // Warpgroup 0 (producer, MMA issuer, two idle warps) gives registers to the
+  // softmax warpgroups: 128 x 72 + 256 x 216 = 384 x 168, the launch's
+  // allocation.
+  if (warp < 4) {
+    setmaxnreg_dec<72>();
+  if (warp == 0) {
+    // -------------------------------------------------------------- producer
+    if (lane == 0) {
+      prefetch_tensormap(&a.map_q);
+      prefetch_tensormap(&a.map_k);
+      prefetch_tensormap(&a.map_v);
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        if (tile[x].nsteps == 0) continue;
+        mbar_arrive_expect_tx(&sm.q_full[x], 128u * D * 2u);
         for (int e = 0; e < 2; ++e) {
-          const int blk = (e == 0 || qb < 0) ? qa : qb;
+          const int blk = (e == 0 || tile[x].qb < 0) ? tile[x].qa : tile[x].qb;
           int t, hp, wp;
           block_coords(g, blk, t, hp, wp);
           for (int c = 0; c < D / 64; ++c)
-            tma_load_5d(&sm.q[c][e * 8192], map_q, &sm.q_full, c * 64, wp * 8, hp * 8, t, bh);
-        }
-        int issued_hi = -1;  // last step whose loads were issued
-        for (int j = 0; j < nsteps; ++j) {
-          const int s = j & 1;
-          if (j >= 2 && !mbar_wait(&sm.kv_empty[s], ((j >> 1) - 1) & 1, abort)) {
-            fail(a.status, &sm.abort, kDevErrTimeoutLoad);
-            break;
-          }
-          if (*abort) break;
-          if (j == 0 && (a.debug_flags & SA_DEBUG_STALL_LOADER)) continue;
-          const int nblk = (n_u - 2 * j) >= 2 ? 2 : 1;
-          mbar_arrive_expect_tx(&sm.kv_full[s], uint32_t(nblk) * 2u * 64u * D * 2u);
-          for (int e = 0; e < nblk; ++e) {
-            int kb = list[2 * j + e] & kEntryBlockMask;
-            if (kb >= g.nb) {
-              atomicOr(a.status, kDevErrBadIndex);
-              kb = 0;
-            }
-            int t, hp, wp;
-            block_coords(g, kb, t, hp, wp);
-            for (int c = 0; c < D / 64; ++c) {
-              tma_load_5d(&sm.k[s][c][e * 8192], map_k, &sm.kv_full[s], c * 64, wp * 8, hp * 8, t,
-                          bh);
-              tma_load_5d(&sm.v[s][c][e * 8192], map_v, &sm.kv_full[s], c * 64, wp * 8, hp * 8, t,
-                          bh);
-            }
-          }
-          issued_hi = j;
-        }
-        if (*abort) {
-          // let this CTA's own copies land before the CTA can exit (the wait
-          // ignores the abort flag but is still time-bounded)
-          int never = 0;
-          for (int j = (issued_hi > 0 ? issued_hi - 1 : 0); j <= issued_hi; ++j)
-            mbar_wait(&sm.kv_full[j & 1], (j >> 1) & 1, &never);
+            tma_load_5d(&sm.q[x][c][e * 8192], &a.map_q, &sm.q_full[x], c * 64, wp * 8, hp * 8,
+                        t, bh);
         }
       }
-    } else if (warp == 1) {
-      // ------------------------------------------------------------ MMA issuer
-      if (lane == 0) {
-        const uint32_t id_s2 = idesc_bf16_f32(128, 128, 0, 0);
-        const uint32_t id_s1 = idesc_bf16_f32(128, 64, 0, 0);
-        const uint32_t id_pv = idesc_bf16_f32(128, D, 0, 1);
-        const uint32_t q_addr = smem_u32(&sm.q[0][0]);
-        bool ok = mbar_wait(&sm.q_full, 0, abort);
-        auto issue_s = [&](int j) {
-          const int s = j & 1;
-          const int nblk = (n_u - 2 * j) >= 2 ? 2 : 1;
-          const uint32_t k_addr = smem_u32(&sm.k[s][0][0]);
-          const uint32_t d_tmem = tmem + (s ? kColS1 : kColS0);
+      OpIter it(tile[0].nsteps, tile[1].nsteps);
+      int kind, x, step, k = 0;
+      while (it.next(kind, x, step)) {
+        const int s = k % kSlots, use = k / kSlots;
+        if (use > 0 && !mbar_wait(&sm.empty[s], (use - 1) & 1, abort)) {
+          fail(a.status, &sm.abort, kDevErrTimeoutLoad);
+          break;
+        }
+        if (*abort) break;
+        if (k == 0 && (a.debug_flags & SA_DEBUG_STALL_LOADER)) {
+          ++k;  // test hook: never fill the first slot
+          continue;
+        }
+        const Tile t = x ? tile[1] : tile[0];
+        const int nblk = step_blocks(t, step);
+        mbar_arrive_expect_tx(&sm.full[s], uint32_t(nblk) * 64u * D * 2u);
+        const CUtensorMap* map = kind == 0 ? &a.map_k : &a.map_v;
+        for (int e = 0; e < nblk; ++e) {
+          int kb = t.list[2 * step + e] & kEntryBlockMask;
+          if (kb >= g.nb) {
+            atomicOr(a.status, kDevErrBadIndex);
+            kb = 0;
+          }
+          int tt, hp, wp;
+          block_coords(g, kb, tt, hp, wp);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_5d(&sm.slot[s][c][e * 8192], map, &sm.full[s], c * 64, wp * 8, hp * 8, tt,
+                        bh);
+        }
+        ++k;
+      }
+      if (*abort) {
+        // let this CTA's own copies land before it can exit (time-bounded,
+        // ignoring the abort flag)
+        int never = 0;
+        for (int kk = (k > kSlots ? k - kSlots : 0); kk < k; ++kk) {
+          if (kk == 0 && (a.debug_flags & SA_DEBUG_STALL_LOADER)) continue;
+          mbar_wait(&sm.full[kk % kSlots], (kk / kSlots) & 1, &never);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t id_s2 = idesc_bf16_f32(128, 128, 0, 0);
+      const uint32_t id_s1 = idesc_bf16_f32(128, 64, 0, 0);
+      const uint32_t id_pv = idesc_bf16_f32(128, D, 0, 1);
+      bool q_ready[2] = {false, false};
+      bool ok = true;
+      OpIter it(tile[0].nsteps, tile[1].nsteps);
+      int kind, x, step, k = 0;
+      while (ok && it.next(kind, x, step)) {
+        const int s = k % kSlots, use = k / kSlots;
+        const Tile t = x ? tile[1] : tile[0];
+        const int nblk = step_blocks(t, step);
+        if (kind == 0) {
+          if (!q_ready[x]) {
+            ok = mbar_wait(&sm.q_full[x], 0, abort);
+            if (!ok) break;
+            q_ready[x] = true;
+          }
+          ok = mbar_wait(&sm.full[s], use & 1, abort);
+          if (!ok) break;
+          tc_fence_after_sync();
+          const uint32_t q_addr = smem_u32(&sm.q[x][0][0]);
+          const uint32_t k_addr = smem_u32(&sm.slot[s][0][0]);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = uint32_t(kk >> 2) * kChunkBytes + uint32_t(kk & 3) * 32u;
-            mma_ss(d_tmem, sw128_desc(q_addr + off, 16, 1024), sw128_desc(k_addr + off, 16, 1024),
-                   nblk == 2 ? id_s2 : id_s1, kk > 0);
+            mma_ss(tmem + col_s(x), sw128_desc(q_addr + off, 16, 1024),
+                   sw128_desc(k_addr + off, 16, 1024), nblk == 2 ? id_s2 : id_s1, kk > 0);
           }
-          mma_commit(&sm.s_full[s]);
-        };
-        if (ok) ok = mbar_wait(&sm.kv_full[0], 0, abort);
-        if (ok) {
-          tc_fence_after_sync();
-          issue_s(0);
-        }
-        for (int j = 0; ok && j < nsteps; ++j) {
-          if (j + 1 < nsteps) {
-            ok = mbar_wait(&sm.kv_full[(j + 1) & 1], ((j + 1) >> 1) & 1, abort);
-            if (!ok) break;
-            tc_fence_after_sync();
-            issue_s(j + 1);
-          }
-          ok = mbar_wait(&sm.p_full[j & 1], (j >> 1) & 1, abort);
-          if (!ok) break;
-          tc_fence_after_sync();
-          const int s = j & 1;
-          const int nblk = (n_u - 2 * j) >= 2 ? 2 : 1;
-          const uint32_t v_addr = smem_u32(&sm.v[s][0][0]);
-          const uint32_t p_tmem = tmem + (s ? kColS1 : kColS0);
-          for (int kk = 0; kk < 4 * nblk; ++kk)
-            mma_ts(tmem + kColO, p_tmem + uint32_t(kk) * 8u,
-                   sw128_desc(v_addr + uint32_t(kk) * 2048u, kChunkBytes, 1024), id_pv,
-                   (j > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&sm.pv_done);
-          mma_commit(&sm.kv_empty[s]);
-        }
-        if (ok) {
-          mma_commit(&sm.o_final);
+          mma_commit(&sm.empty[s]);
+          mma_commit(&sm.s_full[x]);
         } else {
-          fail(a.status, &sm.abort, kDevErrTimeoutMma);
-          mma_commit(&sm.drain);  // wait for this thread's in-flight MMAs
-          int never = 0;
-          mbar_wait(&sm.drain, 0, &never);
-        }
-      }
-    } else {
-      // ------------------------------------------------------------ softmax
-      const int quad = warp & 3;
-      const int r = quad * 32 + lane;  // tile row == TMEM lane
-      const int half = r >> 6;
-      const bool row_valid = half == 0 || qb >= 0;
-      const int keep_bit = half ? kEntryKeepB : kEntryKeepA;
-      const uint32_t t_lane = tmem + (uint32_t(quad * 32) << 16);
-      const float sl2 = a.scale_log2;
-      float m = -INFINITY, l = 0.f;
-      bool ok = true;
-      for (int j = 0; j < nsteps; ++j) {
-        const int s = j & 1;
-        const int nblk = (n_u - 2 * j) >= 2 ? 2 : 1;
-        const int e0 = list[2 * j];
-        const int e1 = nblk == 2 ? list[2 * j + 1] : 0;
-        const bool keep0 = row_valid && (e0 & keep_bit);
-        const bool keep1 = row_valid && nblk == 2 && (e1 & keep_bit);
-        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sm.s_full[s], (j >> 1) & 1, abort));
-        if (!ok) break;
-        tc_fence_after_sync();
-        const uint32_t s_col = t_lane + (s ? kColS1 : kColS0);
-        uint32_t sv[128];
-        tmem_ld32(s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        if (nblk == 2) {
-          tmem_ld32(s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
-          tmem_ld32(s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
-        }
-        tmem_wait_ld();
-        float mx = -INFINITY;
-        if (keep0) {
-#pragma unroll
-          for (int i = 0; i < 64; ++i) mx = fmaxf(mx, __uint_as_float(sv[i]));
-        }
-        if (keep1) {
-#pragma unroll
-          for (int i = 64; i < 128; ++i) mx = fmaxf(mx, __uint_as_float(sv[i]));
-        }
-        mx *= sl2;
-        const bool need = mx > m + kRescaleThreshold;  // false while mx = -inf
-        const float m_new = need ? mx : m;
-        const float alpha = need ? ex2_approx(m - m_new) : 1.f;  // m = -inf -> 0
-        if (__any_sync(0xFFFFFFFFu, need) && j > 0) {
-          ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sm.pv_done, (j - 1) & 1, abort));
+          ok = mbar_wait(&sm.p_full[x], step & 1, abort);
+          if (!ok) break;
+          ok = mbar_wait(&sm.full[s], use & 1, abort);
           if (!ok) break;
           tc_fence_after_sync();
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(t_lane + kColO + 32 * c, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(t_lane + kColO + 32 * c, o);
-          }
+          const uint32_t v_addr = smem_u32(&sm.slot[s][0][0]);
+          for (int kk = 0; kk < 4 * nblk; ++kk)
+            mma_ts(tmem + col_o(x), tmem + col_s(x) + uint32_t(kk) * 8u,
+                   sw128_desc(v_addr + uint32_t(kk) * 2048u, kChunkBytes, 1024), id_pv,
+                   (step > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&sm.empty[s]);
+          if (step == t.nsteps - 1) mma_commit(&sm.o_final[x]);
         }
-        m = m_new;
-        l *= alpha;
-        const float neg_m = -m;
-        float rs = 0.f;
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          float p0 = 0.f, p1 = 0.f;
-          const int base = 2 * i;
-          const bool kp = base < 64 ? keep0 : keep1;
-          if (kp) {
-            p0 = ex2_approx(fmaf(__uint_as_float(sv[base]), sl2, neg_m));
-            p1 = ex2_approx(fmaf(__uint_as_float(sv[base + 1]), sl2, neg_m));
-          }
-          rs += p0 + p1;
-          sv[i] = pack_bf16x2(p0, p1);
-        }
-        l += rs;
-        tmem_st32(s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        if (nblk == 2) tmem_st32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        tmem_wait_st();
-        tc_fence_before_sync();
-        mbar_arrive(&sm.p_full[s]);
+        ++k;
       }
       if (!ok) {
+        fail(a.status, &sm.abort, kDevErrTimeoutMma);
+        mma_commit(&sm.drain);  // wait for this thread's in-flight MMAs
+        int never = 0;
+        mbar_wait(&sm.drain, 0, &never);
+      }
+    }
+  }
+  } else {
+    setmaxnreg_inc<216>();
+    // -------------------------------------------------------------- softmax
+    const int x = (warp - 4) >> 2;  // 0: tile A, 1: tile B
+    const Tile t = x ? tile[1] : tile[0];
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;  // tile row == TMEM lane
+    const int half = r >> 6;
+    const bool row_valid = t.nsteps > 0 && (half == 0 || t.qb >= 0);
+    const int keep_bit = half ? kEntryKeepB : kEntryKeepA;
+    const uint32_t t_lane = tmem + (uint32_t(quad * 32) << 16);
+    const uint32_t s_col = t_lane + col_s(x);
+    const uint32_t o_col = t_lane + col_o(x);
+    const float sl2 = a.scale_log2;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < t.nsteps; ++j) {
+      const int nblk = step_blocks(t, j);
+      const int e0 = t.list[2 * j];
+      const int e1 = nblk == 2 ? t.list[2 * j + 1] : 0;
+      const bool keep0 = row_valid && (e0 & keep_bit);
+      const bool keep1 = row_valid && nblk == 2 && (e1 & keep_bit);
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sm.s_full[x], j & 1, abort));
+      if (!ok) break;
+      tc_fence_after_sync();
+      // keep0 / keep1 are uniform across a warp (a warp's rows lie in one
+      // q-block), so the warp-collective loads may be skipped per block
+      uint32_t sv[128];
+      if (keep0) {
+        tmem_ld32(s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+      }
+      if (keep1) {
+        tmem_ld32(s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
+        tmem_ld32(s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+      }
+      tmem_wait_ld();
+      float mx = -INFINITY;
+      if (keep0) {
+#pragma unroll
+        for (int i = 0; i < 64; i += 2)
+          mx = max3(mx, __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
+      }
+      if (keep1) {
+#pragma unroll
+        for (int i = 64; i < 128; i += 2)
+          mx = max3(mx, __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
+      }
+      mx *= sl2;
+      const bool need = mx > m + kRescaleThreshold;  // false while mx = -inf
+      const float m_new = need ? mx : m;
+      const float alpha = need ? ex2_approx(m - m_new) : 1.f;  // m = -inf -> 0
+      if (__any_sync(0xFFFFFFFFu, need) && j > 0) {
+        // PV_X(j-1) was issued before S_X(j): it is complete here.
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(o_col + 32 * c, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(o_col + 32 * c, o);
+        }
+      }
+      m = m_new;
+      l *= alpha;
+      // p = 2^(s * log2(e)/sqrt(d) - m), two columns per packed op; 3 of every
+      // 8 column pairs take the FMA-pipe exp2, the rest the SFU's ex2.
+      const uint64_t sl2x2 = f2_pack(sl2, sl2);
+      const uint64_t negm2 = f2_pack(-m, -m);
+      uint64_t rs2 = f2_pack(0.f, 0.f);
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        const bool kp = (2 * i) < 64 ? keep0 : keep1;
+        uint32_t packed = 0u;
+        if (kp) {
+          const uint64_t x2 =
+              f2_fma(f2_pack(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), sl2x2,
+                     negm2);
+          float x0, x1;
+          f2_unpack(x2, x0, x1);
+          uint64_t e2;
+          if ((i & 7) >= 5) {
+            e2 = exp2_poly_x2(f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f)));
+          } else {
+            e2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+          }
+          rs2 = f2_add(rs2, e2);
+          float p0, p1;
+          f2_unpack(e2, p0, p1);
+          packed = pack_bf16x2(p0, p1);
+        }
+        sv[i] = packed;
+      }
+      float rs_lo, rs_hi;
+      f2_unpack(rs2, rs_lo, rs_hi);
+      const float rs = rs_lo + rs_hi;
+      l += rs;
+      tmem_st32(s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      if (nblk == 2) tmem_st32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+      tmem_wait_st();
+      tc_fence_before_sync();
+      mbar_arrive(&sm.p_full[x]);
+    }
+    if (t.nsteps > 0) {
+      if (!ok) {
         fail(a.status, &sm.abort, kDevErrTimeoutSoftmax);
-      } else if (__all_sync(0xFFFFFFFFu, mbar_wait(&sm.o_final, 0, abort))) {
+      } else if (__all_sync(0xFFFFFFFFu, mbar_wait(&sm.o_final[x], 0, abort))) {
         tc_fence_after_sync();
         // ---- epilogue: O / l -> natural token position
-        const int blk = half ? qb : qa;
         if (row_valid) {
-          int t, hp, wp;
-          block_coords(g, blk, t, hp, wp);
+          const int blk = half ? t.qb : t.qa;
+          int tt, hp, wp;
+          block_coords(g, blk, tt, hp, wp);
           const int i = r & 63;
-          const size_t tok = size_t(t) * g.Hh * g.Ww + size_t(hp * 8 + (i >> 3)) * g.Ww +
+          const size_t tok = size_t(tt) * g.Hh * g.Ww + size_t(hp * 8 + (i >> 3)) * g.Ww +
                              size_t(wp * 8 + (i & 7));
           const size_t row = size_t(bh) * g.S + tok;
           const float inv = l > 0.f ? 1.0f / l : 0.f;
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
-            tmem_ld32(t_lane + kColO + 32 * c, o);
+            tmem_ld32(o_col + 32 * c, o);
             tmem_wait_ld();
             if (a.out_fp32) {
-              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + row * D + 32 * c);
+              float4* dst =
+                  reinterpret_cast<float4*>(static_cast<float*>(a.out) + row * D + 32 * c);
 #pragma unroll
               for (int v4 = 0; v4 < 8; ++v4)
                 dst[v4] = make_float4(__uint_as_float(o[4 * v4]) * inv,
@@ -352,12 +470,12 @@ template <int D>
 static cudaError_t launch_attn_d(const AttnArgs& a, const Geometry& g, cudaStream_t stream) {
   // At least 120 KB so that one CTA occupies an SM: each CTA allocates all
   // 512 TMEM columns.
-  const size_t smem = sizeof(AttnSmem<D>) + 1024 > 120 * 1024 ? sizeof(AttnSmem<D>) + 1024
-                                                               : 120 * 1024;
+  const size_t need = sizeof(AttnSmem<D>) + 1024;
+  const size_t smem = need > 120 * 1024 ? need : 120 * 1024;
   cudaError_t e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        int(smem));
   if (e != cudaSuccess) return e;
-  const dim3 grid(unsigned(g.ntile), unsigned(g.BH));
+  const dim3 grid(unsigned((g.ntile + 1) / 2), unsigned(g.BH));
   attn_kernel<D><<<grid, kThreads, smem, stream>>>(a, g);
   return cudaGetLastError();
 }

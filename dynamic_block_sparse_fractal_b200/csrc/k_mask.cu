@@ -291,4 +291,46 @@ cudaError_t launch_mask(const MaskArgs& a, const Geometry& g, cudaStream_t strea
   return cudaGetLastError();
 }
 
+// One CTA per head: bitonic sort of the head's tiles by descending union
+// length, so that the attention grid meets the heaviest tiles of a head first
+// (longest-processing-time order) while concurrently running CTAs still share
+// one head's K/V in L2.
+__global__ void __launch_bounds__(1024) tile_order_kernel(const int32_t* __restrict__ tcnt,
+                                                          int32_t* __restrict__ order, Geometry g) {
+  __shared__ uint32_t key[2048];
+  const int bh = blockIdx.x;
+  int n = 1;
+  while (n < g.ntile) n <<= 1;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    // ascending key = descending count, then ascending tile; padding sorts last
+    key[i] = i < g.ntile ? (uint32_t(g.nb - tcnt[size_t(bh) * g.ntile + i]) << 16) | uint32_t(i)
+                         : 0xFFFFFFFFu;
+  }
+  __syncthreads();
+  for (int size = 2; size <= n; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int partner = i ^ stride;
+        if (partner > i) {
+          const bool up = (i & size) == 0;
+          const uint32_t a = key[i], b = key[partner];
+          if ((a > b) == up) {
+            key[i] = b;
+            key[partner] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = threadIdx.x; i < g.ntile; i += blockDim.x)
+    order[size_t(bh) * g.ntile + i] = int32_t(key[i] & 0xFFFFu);
+}
+
+cudaError_t launch_tile_order(const int32_t* tcnt, int32_t* order, const Geometry& g,
+                              cudaStream_t stream) {
+  tile_order_kernel<<<unsigned(g.BH), 1024, 0, stream>>>(tcnt, order, g);
+  return cudaGetLastError();
+}
+
 }  // namespace sa

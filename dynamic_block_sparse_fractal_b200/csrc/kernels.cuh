@@ -35,11 +35,16 @@ struct MaskArgs {
 cudaError_t launch_mask(const MaskArgs& a, const Geometry& g, cudaStream_t stream);
 size_t mask_smem_bytes(const Geometry& g);
 
+// Per head: tiles sorted by descending union length (ties by tile index).
+cudaError_t launch_tile_order(const int32_t* tcnt, int32_t* order, const Geometry& g,
+                              cudaStream_t stream);
+
 struct AttnArgs {
   CUtensorMap map_q, map_k, map_v;  // 5-D patch maps, see tma_host.h
   void* out;
   const int32_t* tcnt;
   const int32_t* tidx;
+  const int32_t* order;
   uint32_t* status;
   float scale_log2;  // log2(e) / sqrt(d)
   int out_fp32;

@@ -73,6 +73,7 @@ struct WsLayout {
   size_t idx;      // int32 [BH][nb][nb]
   size_t tcnt;     // int32 [BH][ntile]
   size_t tidx;     // int32 [BH][ntile][nb]
+  size_t order;    // int32 [BH][ntile]: tiles of a head, heaviest union first
   size_t total;
 };
 
@@ -88,6 +89,7 @@ inline WsLayout make_ws_layout(const Geometry& g) {
   w.idx = o; o = align256(o + sizeof(int32_t) * size_t(g.BH) * g.nb * g.nb);
   w.tcnt = o; o = align256(o + sizeof(int32_t) * size_t(g.BH) * g.ntile);
   w.tidx = o; o = align256(o + sizeof(int32_t) * size_t(g.BH) * g.ntile * g.nb);
+  w.order = o; o = align256(o + sizeof(int32_t) * size_t(g.BH) * g.ntile);
   w.total = o;
   return w;
 }
