@@ -11,9 +11,9 @@
 // heaviest-first tile order), so that the tensor core works on one tile while
 // the softmax warps of the other run:
 //
-//   warp 0      TMA producer: the two Q tiles, then one 32 KB ring slot per
-//               MMA (a K pair for S, a V pair for PV) in exactly the order the
-//               MMA warp consumes them. Q/K/V are read in natural layout
+//   producers   the two Q tiles, then one 32 KB ring slot per MMA (a K pair
+//               for S, a V pair for PV) in exactly the order the MMA warp
+//               consumes them. Q/K/V are read in natural layout
 //               through 5-D tensor maps whose box is one 8x8 patch of one
 //               frame, so the fractal flattening is pure addressing.
 //   warp 1      owns TMEM (S_A, S_B, O_A, O_B: 4 x 128 columns) and issues
@@ -26,7 +26,8 @@
 //               domain, P written back as bf16 over S in TMEM, O rescaled in
 //               TMEM only when the running max grows by more than 2^8 (exact
 //               after the final 1/l), epilogue O / l -> natural token position.
-//   warps 2-3   idle.
+//   warps 0,2,3 TMA producers (every third op each): one issuing thread
+//               keeps too few boxes in flight to feed the tensor core.
 //
 // Ordering facts the pipeline relies on: tcgen05.mma ops issued by one thread
 // execute in order, and a tcgen05.commit tracks every op issued before it. So
@@ -49,9 +50,14 @@ namespace {
 
 constexpr int kThreads = 384;
 constexpr int kSlots = 4;
+constexpr int kProducers = 3;  // TMA-issuing warps (0, 2, 3)
 constexpr int kChunkBytes = 128 * 128;  // 128 rows x 128 B (64 bf16 channels)
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Column pairs (of every 8) whose exp2 runs on the FMA pipe instead of the
+// SFU. Measured on the HunyuanVideo-like workload: the SFU is not yet the
+// limit, and 3 of 8 made the softmax 1.7x slower, so all go to the SFU.
+constexpr int kPolyPairsPer8 = 0;
 constexpr int kMaxList = 2880;             // largest union: nb <= 2880 blocks
 
 __host__ __device__ constexpr uint32_t col_s(int x) { return uint32_t(x) * 128u; }
@@ -183,33 +189,42 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = sm.tmem_base;
 
-  // Warpgroup 0 (producer, MMA issuer, two idle warps) gives registers to the
+  // Warpgroup 0 (three producers and the MMA issuer) gives registers to the
   // softmax warpgroups: 128 x 72 + 256 x 216 = 384 x 168, the launch's
   // allocation.
   if (warp < 4) {
     setmaxnreg_dec<72>();
-  if (warp == 0) {
-    // -------------------------------------------------------------- producer
+  if (warp != 1) {
+    // -------------------------------------------------------------- producers
+    // Warps 0, 2 and 3 each issue every third op's TMA loads: a single
+    // issuing thread cannot keep enough boxes in flight to feed the MMAs.
+    const int prod = warp == 0 ? 0 : warp - 1;  // 0, 1, 2
     if (lane == 0) {
-      prefetch_tensormap(&a.map_q);
-      prefetch_tensormap(&a.map_k);
-      prefetch_tensormap(&a.map_v);
+      if (prod == 0) {
+        prefetch_tensormap(&a.map_q);
+        prefetch_tensormap(&a.map_k);
+        prefetch_tensormap(&a.map_v);
 #pragma unroll
-      for (int x = 0; x < 2; ++x) {
-        if (tile[x].nsteps == 0) continue;
-        mbar_arrive_expect_tx(&sm.q_full[x], 128u * D * 2u);
-        for (int e = 0; e < 2; ++e) {
-          const int blk = (e == 0 || tile[x].qb < 0) ? tile[x].qa : tile[x].qb;
-          int t, hp, wp;
-          block_coords(g, blk, t, hp, wp);
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_5d(&sm.q[x][c][e * 8192], &a.map_q, &sm.q_full[x], c * 64, wp * 8, hp * 8,
-                        t, bh);
+        for (int x = 0; x < 2; ++x) {
+          if (tile[x].nsteps == 0) continue;
+          mbar_arrive_expect_tx(&sm.q_full[x], 128u * D * 2u);
+          for (int e = 0; e < 2; ++e) {
+            const int blk = (e == 0 || tile[x].qb < 0) ? tile[x].qa : tile[x].qb;
+            int t, hp, wp;
+            block_coords(g, blk, t, hp, wp);
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_5d(&sm.q[x][c][e * 8192], &a.map_q, &sm.q_full[x], c * 64, wp * 8, hp * 8,
+                          t, bh);
+          }
         }
       }
       OpIter it(tile[0].nsteps, tile[1].nsteps);
-      int kind, x, step, k = 0;
+      int kind, x, step, k = 0, last_issued = -1;
       while (it.next(kind, x, step)) {
+        if (k % kProducers != prod) {
+          ++k;
+          continue;
+        }
         const int s = k % kSlots, use = k / kSlots;
         if (use > 0 && !mbar_wait(&sm.empty[s], (use - 1) & 1, abort)) {
           fail(a.status, &sm.abort, kDevErrTimeoutLoad);
@@ -236,16 +251,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_5d(&sm.slot[s][c][e * 8192], map, &sm.full[s], c * 64, wp * 8, hp * 8, tt,
                         bh);
         }
+        last_issued = k;
         ++k;
       }
-      if (*abort) {
-        // let this CTA's own copies land before it can exit (time-bounded,
-        // ignoring the abort flag)
+      if (*abort && last_issued >= 0) {
+        // let this warp's own copies land before the CTA can exit
+        // (time-bounded, ignoring the abort flag); at most one op per slot
+        // can still be in flight
         int never = 0;
-        for (int kk = (k > kSlots ? k - kSlots : 0); kk < k; ++kk) {
-          if (kk == 0 && (a.debug_flags & SA_DEBUG_STALL_LOADER)) continue;
+        for (int kk = last_issued; kk >= 0 && kk > last_issued - kSlots; kk -= kProducers)
           mbar_wait(&sm.full[kk % kSlots], (kk / kSlots) & 1, &never);
-        }
       }
     }
   } else if (warp == 1) {
@@ -371,8 +386,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       m = m_new;
       l *= alpha;
-      // p = 2^(s * log2(e)/sqrt(d) - m), two columns per packed op; 3 of every
-      // 8 column pairs take the FMA-pipe exp2, the rest the SFU's ex2.
+      // p = 2^(s * log2(e)/sqrt(d) - m), two columns per packed op;
+      // kPolyPairsPer8 of every 8 column pairs take the FMA-pipe exp2.
       const uint64_t sl2x2 = f2_pack(sl2, sl2);
       const uint64_t negm2 = f2_pack(-m, -m);
       uint64_t rs2 = f2_pack(0.f, 0.f);
@@ -387,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float x0, x1;
           f2_unpack(x2, x0, x1);
           uint64_t e2;
-          if ((i & 7) >= 5) {
+          if ((i & 7) >= 8 - kPolyPairsPer8) {
             e2 = exp2_poly_x2(f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f)));
           } else {
             e2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
