@@ -124,7 +124,9 @@ sa_status sparse_attn_fwd(const sa_desc* desc, const void* q, const void* k, con
   std::memset(&a, 0, sizeof(a));
   if (!encode_patch_map(&a.map_q, q, g.BH, g.T, g.Hh, g.Ww, g.d, g.P) ||
       !encode_patch_map(&a.map_k, k, g.BH, g.T, g.Hh, g.Ww, g.d, g.P) ||
-      !encode_patch_map(&a.map_v, v, g.BH, g.T, g.Hh, g.Ww, g.d, g.P))
+      !encode_patch_map(&a.map_v, v, g.BH, g.T, g.Hh, g.Ww, g.d, g.P) ||
+      !encode_patch_map(&a.map_k2, k, g.BH, g.T, g.Hh, g.Ww, g.d, g.P, g.T > 1 ? 2 : 1) ||
+      !encode_patch_map(&a.map_v2, v, g.BH, g.T, g.Hh, g.Ww, g.d, g.P, g.T > 1 ? 2 : 1))
     return SA_ERR_CUDA;
   a.out = out;
   a.tcnt = at<int32_t>(workspace, w.tcnt);

@@ -204,6 +204,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tensormap(&a.map_q);
         prefetch_tensormap(&a.map_k);
         prefetch_tensormap(&a.map_v);
+        prefetch_tensormap(&a.map_k2);
+        prefetch_tensormap(&a.map_v2);
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
           if (tile[x].nsteps == 0) continue;
@@ -238,18 +240,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Tile t = x ? tile[1] : tile[0];
         const int nblk = step_blocks(t, step);
         mbar_arrive_expect_tx(&sm.full[s], uint32_t(nblk) * 64u * D * 2u);
-        const CUtensorMap* map = kind == 0 ? &a.map_k : &a.map_v;
-        for (int e = 0; e < nblk; ++e) {
-          int kb = t.list[2 * step + e] & kEntryBlockMask;
-          if (kb >= g.nb) {
-            atomicOr(a.status, kDevErrBadIndex);
-            kb = 0;
-          }
+        const int e0 = t.list[2 * step];
+        if (nblk == 2 && (e0 & kEntryTPair) && (e0 & kEntryBlockMask) + g.nh * g.nw < g.nb) {
+          // the same patch in frames t, t+1: one two-frame box per channel half
           int tt, hp, wp;
-          block_coords(g, kb, tt, hp, wp);
+          block_coords(g, e0 & kEntryBlockMask, tt, hp, wp);
+          const CUtensorMap* map = kind == 0 ? &a.map_k2 : &a.map_v2;
           for (int c = 0; c < D / 64; ++c)
-            tma_load_5d(&sm.slot[s][c][e * 8192], map, &sm.full[s], c * 64, wp * 8, hp * 8, tt,
-                        bh);
+            tma_load_5d(&sm.slot[s][c][0], map, &sm.full[s], c * 64, wp * 8, hp * 8, tt, bh);
+        } else {
+          const CUtensorMap* map = kind == 0 ? &a.map_k : &a.map_v;
+          for (int e = 0; e < nblk; ++e) {
+            int kb = t.list[2 * step + e] & kEntryBlockMask;
+            if (kb >= g.nb) {
+              atomicOr(a.status, kDevErrBadIndex);
+              kb = 0;
+            }
+            int tt, hp, wp;
+            block_coords(g, kb, tt, hp, wp);
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_5d(&sm.slot[s][c][e * 8192], map, &sm.full[s], c * 64, wp * 8, hp * 8, tt,
+                          bh);
+          }
         }
         last_issued = k;
         ++k;

@@ -16,7 +16,7 @@
 //  4. OR with the static STA window, compaction into the ascending kept list
 //     and a keep bitmap per row;
 //  5. per query tile (two rows), the union of the two bitmaps as a list of
-//     k-blocks tagged with which q-block keeps each.
+//     k-blocks tagged with which q-block keeps each, temporal pairs first.
 #include <cuda_runtime.h>
 
 #include "kernels.cuh"
@@ -251,22 +251,64 @@ __global__ void __launch_bounds__(kMaskThreads, 1) mask_kernel(MaskArgs a, Geome
   }
   __syncthreads();
 
-  // ---- 5. per-tile union lists
+  // ---- 5. per-tile union lists, ordered for the attention kernel: first the
+  // steps that pair the same patch in frames t and t+1 (one two-frame TMA box
+  // each), then the remaining blocks in ascending order. The probability
+  // buffer L is free now and holds the pairing bitmaps.
   if (warp < kMaskRows / 2) {
     const int tile = tile0 + warp;
     if (tile < g.ntile) {
       const uint32_t* ba = bits + size_t(2 * warp) * nwords;
       const uint32_t* bb = bits + size_t(2 * warp + 1) * nwords;
+      uint32_t* u = reinterpret_cast<uint32_t*>(L) + size_t(warp) * 3 * nwords;
+      uint32_t* first = u + nwords;
+      uint32_t* second = first + nwords;
+      for (int w = lane; w < nwords; w += 32) {
+        u[w] = ba[w] | bb[w];
+        first[w] = 0u;
+        second[w] = 0u;
+      }
+      __syncwarp();
+      // greedy along time, one patch per lane
+      const int pf = g.nh * g.nw;
+      for (int p = lane; p < pf; p += 32) {
+        bool pending = false;
+        for (int t = 0; t < g.T; ++t) {
+          const int b = t * pf + p;
+          const bool in = (u[b >> 5] >> (b & 31)) & 1u;
+          if (pending && in) {
+            const int f = b - pf;
+            atomicOr(&first[f >> 5], 1u << (f & 31));
+            atomicOr(&second[b >> 5], 1u << (b & 31));
+            pending = false;
+          } else {
+            pending = in;
+          }
+        }
+      }
+      __syncwarp();
       int32_t* out = a.tidx + (size_t(bh) * g.ntile + tile) * nb;
+      auto flags = [&](int b) {
+        return int(((ba[b >> 5] >> (b & 31)) & 1u) << 16) | int(((bb[b >> 5] >> (b & 31)) & 1u) << 17);
+      };
       int pos = 0;
       for (int w = 0; w < nwords; ++w) {
-        const uint32_t xa = ba[w], xb = bb[w], u = xa | xb;
-        if ((u >> lane) & 1u) {
-          const int e = (w * 32 + lane) | int(((xa >> lane) & 1u) << 16) |
-                        int(((xb >> lane) & 1u) << 17);
-          out[pos + __popc(u & lanemask_lt())] = e;
+        const uint32_t x = first[w];
+        if ((x >> lane) & 1u) {
+          const int b = w * 32 + lane;
+          const int o = pos + 2 * __popc(x & lanemask_lt());
+          out[o] = b | flags(b) | kEntryTPair;
+          out[o + 1] = (b + pf) | flags(b + pf);
         }
-        pos += __popc(u);
+        pos += 2 * __popc(x);
+      }
+      for (int w = 0; w < nwords; ++w) {
+        const uint32_t x = u[w] & ~first[w] & ~second[w];
+        if ((x >> lane) & 1u) {
+          const int b = w * 32 + lane;
+          out[pos + __popc(x & lanemask_lt())] = b | flags(b);
+        }
+        pos += __popc(x);
       }
       if (lane == 0) a.tcnt[size_t(bh) * g.ntile + tile] = pos;
     }

@@ -41,6 +41,7 @@ cudaError_t launch_tile_order(const int32_t* tcnt, int32_t* order, const Geometr
 
 struct AttnArgs {
   CUtensorMap map_q, map_k, map_v;  // 5-D patch maps, see tma_host.h
+  CUtensorMap map_k2, map_v2;       // the same with two-frame boxes
   void* out;
   const int32_t* tcnt;
   const int32_t* tidx;

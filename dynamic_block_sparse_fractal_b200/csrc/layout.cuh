@@ -95,9 +95,12 @@ inline WsLayout make_ws_layout(const Geometry& g) {
 }
 
 // Union-list entry: k-block id | keep bit of the tile's first q-block << 16
-// | keep bit of the second q-block << 17.
+// | keep bit of the second q-block << 17 | kEntryTPair on the first entry of
+// a step whose two k-blocks are the same patch in frames t and t+1 (the next
+// entry is then this block + patches per frame).
 constexpr int kEntryBlockMask = 0xFFFF;
 constexpr int kEntryKeepA = 1 << 16;
 constexpr int kEntryKeepB = 1 << 17;
+constexpr int kEntryTPair = 1 << 18;
 
 }  // namespace sa

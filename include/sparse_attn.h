@@ -121,7 +121,11 @@ typedef struct sa_mask_views {
   const int32_t* tile_cnt;  /* [B*H][ntile] union length per query tile */
   const int32_t* tile_idx;  /* [B*H][ntile][nb] union entries: k-block id in
                                bits 0-15, bit 16 = first q-block keeps it,
-                               bit 17 = second q-block keeps it */
+                               bit 17 = second q-block keeps it, bit 18 set on
+                               the first entry of each leading pair of entries
+                               that are one patch in frames t and t+1 (these
+                               pairs come first, then the other blocks in
+                               ascending order) */
   int nb;                /* blocks per head */
   int ntile;             /* query tiles per head (pairs of q-blocks) */
 } sa_mask_views;

@@ -139,9 +139,18 @@ def test_union_lists_match_per_block_lists():
             mb = gm[bh, qb] if qb >= 0 else np.zeros_like(ma)
             ent = ti[bh, t, :tc[bh, t]]
             blocks = ent & 0xFFFF
-            assert np.array_equal(blocks, np.nonzero(ma | mb)[0])
+            assert np.array_equal(np.sort(blocks), np.nonzero(ma | mb)[0])
             assert np.array_equal((ent >> 16) & 1, ma[blocks].astype(np.int32))
             assert np.array_equal((ent >> 17) & 1, mb[blocks].astype(np.int32))
+            # leading temporal pairs (same patch, frames t and t+1), then the
+            # remaining blocks ascending
+            tp = (ent >> 18) & 1
+            npair = int(tp.sum())
+            assert not tp[2 * npair:].any() and tp[0:2 * npair:2].all()
+            pf = (w.Hh // w.P) * (w.Ww // w.P)
+            assert np.array_equal(blocks[1:2 * npair:2], blocks[0:2 * npair:2] + pf)
+            rest = blocks[2 * npair:]
+            assert np.array_equal(rest, np.sort(rest))
 
 
 # ---------------------------------------------------------------- edge shapes
