@@ -277,52 +277,81 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // -------------------------------------------------------------- MMA issuer
+    // One thread issues every MMA; its SMSP is shared with two busy softmax
+    // warps, so the bookkeeping between MMA batches is kept to a minimum
+    // (each instruction here idles the tensor core once its short queue
+    // drains).
     if (lane == 0) {
       const uint32_t id_s2 = idesc_bf16_f32(128, 128, 0, 0);
       const uint32_t id_s1 = idesc_bf16_f32(128, 64, 0, 0);
       const uint32_t id_pv = idesc_bf16_f32(128, D, 0, 1);
-      bool q_ready[2] = {false, false};
-      bool ok = true;
-      OpIter it(tile[0].nsteps, tile[1].nsteps);
-      int kind, x, step, k = 0;
-      while (ok && it.next(kind, x, step)) {
-        const int s = k % kSlots, use = k / kSlots;
-        const Tile t = x ? tile[1] : tile[0];
-        const int nblk = step_blocks(t, step);
-        if (kind == 0) {
-          if (!q_ready[x]) {
-            ok = mbar_wait(&sm.q_full[x], 0, abort);
-            if (!ok) break;
-            q_ready[x] = true;
-          }
-          ok = mbar_wait(&sm.full[s], use & 1, abort);
-          if (!ok) break;
-          tc_fence_after_sync();
-          const uint32_t q_addr = smem_u32(&sm.q[x][0][0]);
-          const uint32_t k_addr = smem_u32(&sm.slot[s][0][0]);
+      // Descriptors differ only in the start-address field (bits 0-13, in
+      // 16-byte units), so each MMA below is one 32-bit add from a base.
+      const uint64_t kdesc0 = sw128_desc(smem_u32(&sm.slot[0][0][0]), 16, 1024);
+      const uint64_t vdesc0 = sw128_desc(smem_u32(&sm.slot[0][0][0]), kChunkBytes, 1024);
+      const uint64_t qdesc0 = sw128_desc(smem_u32(&sm.q[0][0][0]), 16, 1024);
+      const uint64_t qdesc1 = sw128_desc(smem_u32(&sm.q[1][0][0]), 16, 1024);
+      constexpr uint32_t kSlotStep = (D / 64) * kChunkBytes / 16;  // one slot, 16 B units
+      const int n0 = tile[0].nsteps, n1 = tile[1].nsteps;
+      const int u0 = tile[0].n_u, u1 = tile[1].n_u;
+      bool ok = mbar_wait(&sm.q_full[0], 0, abort);
+      if (ok && n1 > 0) ok = mbar_wait(&sm.q_full[1], 0, abort);
+      int k = 0;  // op index (ring position)
+      auto issue_s = [&](int x, int step) {
+        const int s = k & (kSlots - 1);
+        if (!mbar_wait(&sm.full[s], (k / kSlots) & 1, abort)) return false;
+        const uint64_t qd = x ? qdesc1 : qdesc0;
+        const uint64_t kd = kdesc0 + uint64_t(s) * kSlotStep;
+        const uint32_t id = ((x ? u1 : u0) - 2 * step) >= 2 ? id_s2 : id_s1;
+        const uint32_t d_tmem = tmem + col_s(x);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = uint32_t(kk >> 2) * kChunkBytes + uint32_t(kk & 3) * 32u;
-            mma_ss(tmem + col_s(x), sw128_desc(q_addr + off, 16, 1024),
-                   sw128_desc(k_addr + off, 16, 1024), nblk == 2 ? id_s2 : id_s1, kk > 0);
-          }
-          mma_commit(&sm.empty[s]);
-          mma_commit(&sm.s_full[x]);
-        } else {
-          ok = mbar_wait(&sm.p_full[x], step & 1, abort);
-          if (!ok) break;
-          ok = mbar_wait(&sm.full[s], use & 1, abort);
-          if (!ok) break;
-          tc_fence_after_sync();
-          const uint32_t v_addr = smem_u32(&sm.slot[s][0][0]);
-          for (int kk = 0; kk < 4 * nblk; ++kk)
-            mma_ts(tmem + col_o(x), tmem + col_s(x) + uint32_t(kk) * 8u,
-                   sw128_desc(v_addr + uint32_t(kk) * 2048u, kChunkBytes, 1024), id_pv,
-                   (step > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&sm.empty[s]);
-          if (step == t.nsteps - 1) mma_commit(&sm.o_final[x]);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (uint32_t(kk >> 2) * kChunkBytes + uint32_t(kk & 3) * 32u) >> 4;
+          mma_ss(d_tmem, qd + off, kd + off, id, kk > 0);
         }
+        mma_commit(&sm.empty[s]);
+        mma_commit(&sm.s_full[x]);
         ++k;
+        return true;
+      };
+      auto issue_pv = [&](int x, int step) {
+        const int s = k & (kSlots - 1);
+        if (!mbar_wait(&sm.p_full[x], step & 1, abort)) return false;
+        if (!mbar_wait(&sm.full[s], (k / kSlots) & 1, abort)) return false;
+        tc_fence_after_sync();  // P was written by the softmax threads
+        const uint64_t vd = vdesc0 + uint64_t(s) * kSlotStep;
+        const uint32_t o_tmem = tmem + col_o(x);
+        const uint32_t p_tmem = tmem + col_s(x);
+        const uint32_t acc0 = step > 0 ? 1u : 0u;
+        if (((x ? u1 : u0) - 2 * step) >= 2) {
+          mma_ts(o_tmem, p_tmem, vd, id_pv, acc0);
+#pragma unroll
+          for (int kk = 1; kk < 8; ++kk)
+            mma_ts(o_tmem, p_tmem + uint32_t(kk) * 8u, vd + uint32_t(kk) * 128u, id_pv, 1u);
+        } else {
+          mma_ts(o_tmem, p_tmem, vd, id_pv, acc0);
+#pragma unroll
+          for (int kk = 1; kk < 4; ++kk)
+            mma_ts(o_tmem, p_tmem + uint32_t(kk) * 8u, vd + uint32_t(kk) * 128u, id_pv, 1u);
+        }
+        mma_commit(&sm.empty[s]);
+        if (step == (x ? n1 : n0) - 1) mma_commit(&sm.o_final[x]);
+        ++k;
+        return true;
+      };
+      // the order OpIter describes: S_A0 S_B0 | PV_A(j) S_A(j+1) PV_B(j) S_B(j+1) | ...
+      if (ok && n0 > 0) ok = issue_s(0, 0);
+      if (ok && n1 > 0) ok = issue_s(1, 0);
+      const int nmax = n0 > n1 ? n0 : n1;
+      for (int j = 0; ok && j < nmax; ++j) {
+        if (j < n0) {
+          ok = issue_pv(0, j);
+          if (ok && j + 1 < n0) ok = issue_s(0, j + 1);
+        }
+        if (ok && j < n1) {
+          ok = issue_pv(1, j);
+          if (ok && j + 1 < n1) ok = issue_s(1, j + 1);
+        }
       }
       if (!ok) {
         fail(a.status, &sm.abort, kDevErrTimeoutMma);
