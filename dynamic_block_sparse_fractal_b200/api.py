@@ -26,8 +26,9 @@ SA_DEBUG_STALL_LOADER = 1
 SYMBOLS = (
     "sparse_attn_workspace_size", "sparse_attn_plan", "sparse_attn_fwd",
     "sparse_attn_permute", "sparse_attn_get_mask", "sparse_attn_tile_blocks",
-    "sparse_attn_check", "sparse_attn_status_string",
+    "sparse_attn_check", "sparse_attn_forward_noalloc", "sparse_attn_status_string",
 )
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class SaDesc(ctypes.Structure):
@@ -71,10 +72,12 @@ def lib() -> ctypes.CDLL:
         L.sparse_attn_get_mask.argtypes = [dp, vp, sz, ctypes.POINTER(SaMaskViews)]
         L.sparse_attn_tile_blocks.argtypes = [dp, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)]
         L.sparse_attn_check.argtypes = [dp, vp, sz, vp]
+        L.sparse_attn_forward_noalloc.argtypes = [dp, vp, vp, vp, vp, vp]
         L.sparse_attn_status_string.argtypes = [i32]
         L.sparse_attn_status_string.restype = ctypes.c_char_p
-        for name in SYMBOLS[:-1]:
-            getattr(L, name).restype = i32
+        for name in SYMBOLS:
+            if name != "sparse_attn_status_string":
+                getattr(L, name).restype = i32
         _lib = L
     return _lib
 
@@ -155,6 +158,16 @@ def permute(desc: SaDesc, x: torch.Tensor, y: torch.Tensor, inverse: bool = Fals
     _ok(lib().sparse_attn_permute(ctypes.byref(desc), _ptr(x), _ptr(y), int(inverse),
                                   _stream(stream)), "permute")
     return y
+
+
+def forward_noalloc(desc: SaDesc, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                    out: torch.Tensor, stream=None) -> torch.Tensor:
+    """Plan + forward with the library's built-in workspace (for callers that
+    cannot allocate device memory); see include/sparse_attn.h."""
+    _check_qkv(desc, q, k, v)
+    _ok(lib().sparse_attn_forward_noalloc(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v),
+                                          _ptr(out), _stream(stream)), "forward_noalloc")
+    return out
 
 
 def check(desc: SaDesc, workspace: torch.Tensor, stream=None) -> int:

@@ -147,6 +147,39 @@ sa_status sparse_attn_check(const sa_desc* desc, const void* workspace,
 /* Static, NUL-terminated description of a status code. */
 const char* sparse_attn_status_string(sa_status status);
 
+/* Bytes of the workspace built into the library for
+ * sparse_attn_forward_noalloc (64 MiB). */
+#define SA_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/* Plan + forward without a caller-provided workspace. (No counterpart in the
+ * NABLA paper: this exists for the library's users, not for the method.)
+ *
+ * Some callers cannot allocate device memory on their own: a runtime that
+ * owns every byte of GPU memory and hands out only what it planned at start-up,
+ * code on a latency-critical path where cudaMalloc's implicit synchronisation
+ * is not acceptable, or a host program that simply has no allocator for the
+ * device. This call lets them run the whole path with only their own q, k, v
+ * and out buffers: the workspace is a fixed SA_NOALLOC_SCRATCH_BYTES array in
+ * the library's device image (each GPU that loads the library holds one copy
+ * until the process exits). The call allocates nothing.
+ *
+ * q, k, v, out, stream and desc are as for sparse_attn_plan/sparse_attn_fwd.
+ * Returns SA_ERR_WORKSPACE, before launching anything, when the problem's
+ * workspace (sparse_attn_workspace_size) is larger than the built-in array.
+ *
+ * - The first call on a device (with that device current) looks the array's
+ *   device address up once; make that first call before any stream capture.
+ * - All calls on a device share the one array, which keeps the previous
+ *   call's contents (the plan rewrites everything it later reads). Calls whose
+ *   work may overlap on the GPU (different streams, or several threads)
+ *   race on it: serialise them.
+ * - Device-side status (a bounded wait that ran out) lands in the shared
+ *   array and is not reported by this call; use the workspace entry points
+ *   with sparse_attn_check when that status matters. */
+sa_status sparse_attn_forward_noalloc(const sa_desc* desc, const void* q,
+                                      const void* k, const void* v, void* out,
+                                      void* stream);
+
 #ifdef __cplusplus
 }
 #endif
