@@ -14,8 +14,9 @@ using namespace sa;
 
 namespace {
 
-// Largest block count per head the mask kernel's shared memory can hold
-// (16 rows of fp32 probabilities plus keep bitmaps).
+// Largest block count per head: the attention kernel stages a tile's union
+// list (<= nb entries) in shared memory sized for 2880 entries (the select
+// kernel's register-held rows would allow 3072).
 constexpr int kMaxBlocks = 2880;
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -91,14 +92,15 @@ sa_status sparse_attn_plan(const sa_desc* desc, const void* q, const void* k, vo
   MaskArgs m;
   m.qbar = at<float>(workspace, w.qbar);
   m.kbar = at<float>(workspace, w.kbar);
+  m.logits = at<float>(workspace, w.logits);
+  m.bits = at<uint32_t>(workspace, w.bits);
   m.cnt = at<int32_t>(workspace, w.cnt);
   m.idx = at<int32_t>(workspace, w.idx);
   m.tcnt = at<int32_t>(workspace, w.tcnt);
   m.tidx = at<int32_t>(workspace, w.tidx);
-  m.status = at<uint32_t>(workspace, w.status);
   m.dense = desc->thr == 0.0f;
-  // mass threshold 1 - thr in the kernel's 2^-40 fixed point
-  m.target_fx = (unsigned long long)std::llround((1.0 - (double)desc->thr) * 1099511627776.0);
+  // mass threshold 1 - thr in the select kernel's 2^-30 fixed point
+  m.target_fx = (uint32_t)std::llround((1.0 - (double)desc->thr) * 1073741824.0);
   const bool sta = desc->sta_t > 0;
   m.sta_t = sta ? desc->sta_t / 2 : -1;
   m.sta_h = sta ? desc->sta_h / 2 : -1;

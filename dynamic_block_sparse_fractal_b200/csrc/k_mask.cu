@@ -1,22 +1,25 @@
 // Mask build (NABLA, Metodologia 2 "Attenzione Ridotta" + "CDF Thresholding",
-// Metodologia 3 STA union). One CTA handles 16 q-block rows (8 query tiles)
-// of one head, one warp per row:
+// Metodologia 3 STA union), three kernels after the pooling:
 //
-//  1. logits L[r][j] = Qbar[r] . Kbar[j] / sqrt(d) in fp32 FFMA, Kbar streamed
-//     through shared memory in chunks of 64 blocks;
-//  2. row softmax (max, exp, one deterministic warp sum);
-//  3. CDF threshold without sorting: k-block j is kept iff the probability
-//     mass ranked before it is < 1 - thr. With masses in 2^-40 fixed point
-//     (integer sums, so the result is bit-identical run to run), a 4-pass
-//     8-bit radix select over the probabilities' bit patterns finds the
-//     probability tau of the last kept block and the mass strictly above it;
-//     blocks equal to tau are kept in ascending index order while the running
-//     mass stays below the threshold (ties broken by index, as the sorted
-//     definition does);
-//  4. OR with the static STA window, compaction into the ascending kept list
-//     and a keep bitmap per row;
-//  5. per query tile (two rows), the union of the two bitmaps as a list of
-//     k-blocks tagged with which q-block keeps each, temporal pairs first.
+//  logits_kernel  L[bh][r][j] = Qbar[r] . Kbar[j] / sqrt(d) for every pair of
+//                 blocks of a head in fp32 FFMA (register-tiled 128 x 128
+//                 output tiles), stored in the workspace;
+//  select_kernel  one warp per q-block row, the row held in registers:
+//                 softmax, then the CDF threshold without sorting. k-block j
+//                 is kept iff the probability mass ranked before it (descending
+//                 order, ties by index) is < 1 - thr. With masses in 2^-30
+//                 fixed point (integer sums, so the result is bit-identical
+//                 run to run), a bitwise binary search over warp-reduced
+//                 partial sums finds the mass tau of the last kept block; of
+//                 the blocks whose mass equals tau, those that keep the
+//                 running mass below the threshold are kept in ascending index
+//                 order. Then the OR with the static STA window, the ascending
+//                 kept list and the row's keep bitmap;
+//  union_kernel   one warp per query tile (two q-blocks): the union of the
+//                 two bitmaps as a list of k-blocks tagged with which q-block
+//                 keeps each, first the steps that pair one patch in frames t
+//                 and t+1 (one two-frame TMA box each in the attention
+//                 kernel), then the remaining blocks in ascending order.
 #include <cuda_runtime.h>
 
 #include "kernels.cuh"
@@ -24,14 +27,9 @@
 
 namespace sa {
 
-constexpr int kMaskRows = 16;
-constexpr int kMaskThreads = kMaskRows * 32;
-constexpr int kKChunk = 64;
-constexpr unsigned kFull = 0xFFFFFFFFu;
+namespace {
 
-__device__ __forceinline__ unsigned long long mass_fx(float p) {
-  return __float2ull_rn(p * 1099511627776.0f);  // p * 2^40, exact scaling
-}
+constexpr unsigned kFull = 0xFFFFFFFFu;
 
 __device__ __forceinline__ unsigned lanemask_lt() {
   unsigned m;
@@ -39,297 +37,484 @@ __device__ __forceinline__ unsigned lanemask_lt() {
   return m;
 }
 
-__host__ __device__ constexpr size_t mask_region2_bytes(int D) {
-  return (size_t(kKChunk) * (D + 4) * 4 > size_t(kMaskRows) * 256 * 8)
-             ? size_t(kKChunk) * (D + 4) * 4
-             : size_t(kMaskRows) * 256 * 8;
-}
+// ------------------------------------------------------------------ logits
+constexpr int kBM = 128, kBN = 128, kBK = 32, kPad = 4;
+constexpr int kLds = kBM + kPad;  // row pitch of a transposed slice (floats)
+constexpr int kLogitThreads = 256;
+constexpr size_t kLogitSmem = size_t(2) * 2 * kBK * kLds * sizeof(float);  // 67,584 B
 
-size_t mask_smem_bytes(const Geometry& g) {
-  const size_t nwords = (g.nb + 31) / 32;
-  return size_t(kMaskRows) * g.d * 4 + mask_region2_bytes(g.d) + size_t(kMaskRows) * g.nb * 4 +
-         size_t(kMaskRows) * nwords * 4;
-}
-
+// Rows [r0, r0 + 128) x channels [k0, k0 + 32) of a [nb][D] fp32 matrix,
+// 4 float4 per thread; rows past nb read as zeros.
 template <int D>
-__global__ void __launch_bounds__(kMaskThreads, 1) mask_kernel(MaskArgs a, Geometry g) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  constexpr int KP = D + 4;  // padded K-chunk row (conflict-free float4 reads)
-  const int nb = g.nb;
-  const int nwords = (nb + 31) / 32;
-  float* qs = reinterpret_cast<float*>(smem);                      // [16][D]
-  uint8_t* region2 = smem + size_t(kMaskRows) * D * 4;              // K chunk / histograms
-  float* ks = reinterpret_cast<float*>(region2);                    // [64][KP]
-  float* L = reinterpret_cast<float*>(region2 + mask_region2_bytes(D));  // [16][nb]
-  uint32_t* bits = reinterpret_cast<uint32_t*>(L + size_t(kMaskRows) * nb);  // [16][nwords]
-  __shared__ int row_blk[kMaskRows];
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.y;
-  const int tile0 = blockIdx.x * (kMaskRows / 2);
-
-  if (threadIdx.x < kMaskRows) {
-    const int tile = tile0 + threadIdx.x / 2;
-    int blk = -1;
-    if (tile < g.ntile) {
-      int qa, qb;
-      tile_blocks(g, tile, qa, qb);
-      blk = (threadIdx.x & 1) ? qb : qa;
-    }
-    row_blk[threadIdx.x] = blk;
+__device__ __forceinline__ void load_slice(const float* __restrict__ m, int nb, int r0, int k0,
+                                           float4 (&v)[4]) {
+  const int t = threadIdx.x;
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    const int row = (t >> 3) + 32 * s;
+    v[s] = (r0 + row < nb)
+               ? __ldg(reinterpret_cast<const float4*>(m + size_t(r0 + row) * D + k0) + (t & 7))
+               : make_float4(0.f, 0.f, 0.f, 0.f);
   }
+}
+
+// Stores a slice transposed, dst[k][row] (channel-major, padded pitch).
+__device__ __forceinline__ void store_slice(float* dst, const float4 (&v)[4]) {
+  const int t = threadIdx.x;
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    const int row = (t >> 3) + 32 * s, k = 4 * (t & 7);
+    dst[(k + 0) * kLds + row] = v[s].x;
+    dst[(k + 1) * kLds + row] = v[s].y;
+    dst[(k + 2) * kLds + row] = v[s].z;
+    dst[(k + 3) * kLds + row] = v[s].w;
+  }
+}
+
+// CTA = one 128 x 128 tile of one head's nb x nb logits; thread (ty, tx)
+// accumulates 8 x 8 outputs: rows r0 + 8 ty + i, columns c0 + 4 tx + j and
+// c0 + 64 + 4 tx + j (two float4 groups, so that a quarter-warp's shared
+// loads hit distinct banks and its global stores are contiguous).
+// Channel slices of 32 are double-buffered: the next slice is fetched into
+// registers while the current one is multiplied out of shared memory.
+template <int D>
+__global__ void __launch_bounds__(kLogitThreads, 1)
+    logits_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
+                  float* __restrict__ L, Geometry g, int ld, float scale) {
+  extern __shared__ __align__(16) float lsm[];
+  float* As = lsm;                 // [2][kBK][kLds]
+  float* Bs = lsm + 2 * kBK * kLds;  // [2][kBK][kLds]
+  const int bh = blockIdx.z;
+  const int r0 = blockIdx.y * kBM, c0 = blockIdx.x * kBN;
+  const float* qa = qbar + size_t(bh) * g.nb * D;
+  const float* kb = kbar + size_t(bh) * g.nb * D;
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+
+  float4 ra[4], rb[4];
+  load_slice<D>(qa, g.nb, r0, 0, ra);
+  load_slice<D>(kb, g.nb, c0, 0, rb);
+  store_slice(As, ra);
+  store_slice(Bs, rb);
   __syncthreads();
-  for (int i = threadIdx.x; i < kMaskRows * D / 4; i += kMaskThreads) {
-    const int r = i / (D / 4), c = i - r * (D / 4);
-    const int blk = row_blk[r];
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (blk >= 0) v = reinterpret_cast<const float4*>(a.qbar + (size_t(bh) * nb + blk) * D)[c];
-    reinterpret_cast<float4*>(qs)[i] = v;
-  }
-
-  // ---- 1. logits
-  const int r = warp;
-  const float* kbase = a.kbar + size_t(bh) * nb * D;
-  for (int c0 = 0; c0 < nb; c0 += kKChunk) {
-    __syncthreads();
-    for (int i = threadIdx.x; i < kKChunk * D / 4; i += kMaskThreads) {
-      const int row = i / (D / 4), c = i - row * (D / 4);
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (c0 + row < nb) v = reinterpret_cast<const float4*>(kbase + size_t(c0 + row) * D)[c];
-      *reinterpret_cast<float4*>(ks + row * KP + 4 * c) = v;
+  constexpr int kSlices = D / kBK;
+#pragma unroll 1
+  for (int c = 0; c < kSlices; ++c) {
+    const int cur = c & 1;
+    if (c + 1 < kSlices) {
+      load_slice<D>(qa, g.nb, r0, (c + 1) * kBK, ra);
+      load_slice<D>(kb, g.nb, c0, (c + 1) * kBK, rb);
     }
-    __syncthreads();
-    const float* qr = qs + r * D;
-    const float* k0 = ks + lane * KP;
-    const float* k1 = ks + (lane + 32) * KP;
-    float acc0 = 0.f, acc1 = 0.f;
+    const float* A = As + cur * kBK * kLds + ty * 8;
+    const float* Bm = Bs + cur * kBK * kLds + tx * 4;
 #pragma unroll 8
-    for (int dd = 0; dd < D; dd += 4) {
-      const float4 qv = *reinterpret_cast<const float4*>(qr + dd);
-      const float4 x0 = *reinterpret_cast<const float4*>(k0 + dd);
-      const float4 x1 = *reinterpret_cast<const float4*>(k1 + dd);
-      acc0 = fmaf(qv.x, x0.x, acc0);
-      acc0 = fmaf(qv.y, x0.y, acc0);
-      acc0 = fmaf(qv.z, x0.z, acc0);
-      acc0 = fmaf(qv.w, x0.w, acc0);
-      acc1 = fmaf(qv.x, x1.x, acc1);
-      acc1 = fmaf(qv.y, x1.y, acc1);
-      acc1 = fmaf(qv.z, x1.z, acc1);
-      acc1 = fmaf(qv.w, x1.w, acc1);
+    for (int k = 0; k < kBK; ++k) {
+      const float4 a0 = *reinterpret_cast<const float4*>(A + k * kLds);
+      const float4 a1 = *reinterpret_cast<const float4*>(A + k * kLds + 4);
+      const float4 b0 = *reinterpret_cast<const float4*>(Bm + k * kLds);
+      const float4 b1 = *reinterpret_cast<const float4*>(Bm + k * kLds + 64);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
     }
-    if (c0 + lane < nb) L[size_t(r) * nb + c0 + lane] = acc0 * a.scale;
-    if (c0 + lane + 32 < nb) L[size_t(r) * nb + c0 + lane + 32] = acc1 * a.scale;
+    if (c + 1 < kSlices) {
+      store_slice(As + (cur ^ 1) * kBK * kLds, ra);
+      store_slice(Bs + (cur ^ 1) * kBK * kLds, rb);
+    }
+    __syncthreads();
   }
-  __syncthreads();  // region2 is free from here on: histograms
+  float* out = L + size_t(bh) * g.nb * ld;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = r0 + ty * 8 + i;
+    if (r < g.nb) {
+      float* dst = out + size_t(r) * ld + c0 + tx * 4;
+      *reinterpret_cast<float4*>(dst) = make_float4(acc[i][0] * scale, acc[i][1] * scale,
+                                                    acc[i][2] * scale, acc[i][3] * scale);
+      *reinterpret_cast<float4*>(dst + 64) = make_float4(acc[i][4] * scale, acc[i][5] * scale,
+                                                         acc[i][6] * scale, acc[i][7] * scale);
+    }
+  }
+}
 
-  const int blk = row_blk[r];
-  uint32_t* my_bits = bits + size_t(r) * nwords;
-  if (blk >= 0) {
-    float* Lr = L + size_t(r) * nb;
-    // ---- 2. softmax
+// ------------------------------------------------------------------ select
+constexpr int kSelWarps = 8;
+constexpr int kCandCap = 256;    // compacted search window per warp (8 per lane)
+constexpr int kMaxRowWords = 96;  // keep-bitmap words of a row (nb <= 3072)
+
+__device__ __forceinline__ uint32_t warp_sum_u32(uint32_t s) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(kFull, s, o);
+  return s;
+}
+
+// Sum over the warp of the masses >= c; eight independent partial sums keep
+// the adds pipelined. (The sum of the masses > c is the one at c + 1.)
+template <int N>
+__device__ __forceinline__ uint32_t mass_at_least(const uint32_t (&m)[N], uint32_t c) {
+  constexpr int kAcc = N < 8 ? N : 8;
+  uint32_t acc[kAcc];
+#pragma unroll
+  for (int i = 0; i < kAcc; ++i) acc[i] = 0u;
+#pragma unroll
+  for (int i = 0; i < N; ++i) acc[i % kAcc] += m[i] >= c ? m[i] : 0u;
+#pragma unroll
+  for (int w = 1; w < kAcc; w <<= 1)
+#pragma unroll
+    for (int i = 0; i + w < kAcc; i += 2 * w) acc[i] += acc[i + w];
+  return warp_sum_u32(acc[0]);
+}
+
+// VPL = values per lane: column j of the row sits in lane j % 32, slot j / 32.
+template <int VPL>
+__global__ void __launch_bounds__(kSelWarps * 32, VPL <= 32 ? 4 : (VPL <= 64 ? 2 : 1))
+    select_kernel(const float* __restrict__ L, MaskArgs a, Geometry g, int ld) {
+  __shared__ uint32_t cand_all[kSelWarps][kCandCap];
+  __shared__ uint32_t rbits_all[kSelWarps][kMaxRowWords];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long row = long(blockIdx.x) * kSelWarps + warp;
+  if (row >= long(g.BH) * g.nb) return;
+  const int nb = g.nb;
+  const int qb = int(row % nb);
+  const float* Lr = L + size_t(row) * ld;
+  constexpr float kLog2e = 1.4426950408889634f;
+
+  // ---- row softmax; each probability as an integer mass m = p * 2^30
+  uint32_t m[VPL];
+  {
+    float v[VPL];
     float mx = -INFINITY;
-    for (int j = lane; j < nb; j += 32) mx = fmaxf(mx, Lr[j]);
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int j = lane + 32 * i;
+      v[i] = j < nb ? __ldg(Lr + j) : -INFINITY;
+      mx = fmaxf(mx, v[i]);
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+    const float shift = -mx * kLog2e;
     float sum = 0.f;
-    for (int j = lane; j < nb; j += 32) {
-      const float e = expf(Lr[j] - mx);
-      Lr[j] = e;
-      sum += e;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      v[i] = ex2_approx(fmaf(v[i], kLog2e, shift));  // exactly 0 in the padding slots
+      sum += v[i];
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(kFull, sum, o);
-    const float inv = 1.0f / sum;
-    for (int j = lane; j < nb; j += 32) Lr[j] *= inv;
-    __syncwarp();
+    const float to_fx = 1073741824.0f / sum;  // 2^30 / sum
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) m[i] = __float2uint_rn(v[i] * to_fx);
+  }
 
-    // ---- 3. CDF threshold by radix select
-    bool keep_all = a.dense != 0;
-    unsigned tau = 0;
-    unsigned long long keep_ties = 0;
-    if (!keep_all) {
-      const unsigned long long tgt = a.target_fx;
-      unsigned long long* hist = reinterpret_cast<unsigned long long*>(region2) + warp * 256;
-      unsigned prefix = 0, pmask = 0;
-      unsigned long long above = 0;
-      for (int pass = 0; pass < 4; ++pass) {
-        const int shift = 24 - 8 * pass;
-        for (int i = lane; i < 256; i += 32) hist[i] = 0ull;
-        __syncwarp();
-        for (int j = lane; j < nb; j += 32) {
-          const float p = Lr[j];
-          const unsigned key = __float_as_uint(p);
-          if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], mass_fx(p));
-        }
-        __syncwarp();
-        // lane l owns bins 255-8l down to 248-8l
-        unsigned long long h[8], s = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          h[i] = hist[255 - 8 * lane - i];
-          s += h[i];
-        }
-        unsigned long long inc = s;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const unsigned long long v = __shfl_up_sync(kFull, inc, o);
-          if (lane >= o) inc += v;
-        }
-        const unsigned long long pre = above + (inc - s);
-        const bool cross = pre < tgt && tgt <= pre + s;
-        const unsigned bal = __ballot_sync(kFull, cross);
-        if (bal == 0u) {  // total mass below the target (rounding): keep all
+  // ---- CDF threshold. In descending mass order (ties by index), block j is
+  // kept iff the mass ranked before it is < target. tau, the mass of the last
+  // kept block, is the largest x with G(x) = (sum of the masses >= x) >=
+  // target; G does not increase with x. Found as: the leading bit e of tau
+  // by a binary search over bit positions, then the lower bits one by one.
+  // Once e is known only the masses in [2^e, 2^(e+1)) can still move G, so
+  // those (if few) are compacted to shared memory and searched alone, the
+  // masses >= 2^(e+1) entering as a constant. Blocks with mass > tau are
+  // kept, and of those with mass == tau the first
+  // ceil((target - G(tau + 1)) / tau) in index order. Every pass over the
+  // whole row goes through the one loop below (the code stays small).
+  bool keep_all = a.dense != 0;
+  uint32_t tau = 0, keep_ties = 0;
+  if (!keep_all) {
+    const uint32_t tgt = a.target_fx;
+    enum { kTotal, kLead, kAbove, kBits, kTies };
+    int stage = kTotal, lo = 0, hi = 0, mid = 0, b = 0;
+    uint32_t c = 1u, x = 0u;
+    for (;;) {
+      const uint32_t s = mass_at_least<VPL>(m, c);
+      if (stage == kTotal) {
+        if (s < tgt) {  // total mass below the target (rounding): keep all
           keep_all = true;
           break;
         }
-        const int src = __ffs(bal) - 1;
-        int digit = 0;
-        unsigned long long above_new = 0;
-        if (lane == src) {
-          unsigned long long run = pre;
+        uint32_t mmax = 0;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            if (run + h[i] >= tgt) {
-              digit = 255 - 8 * lane - i;
-              above_new = run;
-              break;
-            }
-            run += h[i];
-          }
+        for (int i = 0; i < VPL; ++i) mmax = max(mmax, m[i]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mmax = max(mmax, __shfl_xor_sync(kFull, mmax, o));
+        hi = 31 - __clz(mmax);  // G(2^lo) >= target holds for lo = 0
+        stage = kLead;
+      } else if (stage == kLead) {
+        if (s >= tgt) lo = mid;
+        else hi = mid - 1;
+      } else if (stage == kAbove) {
+        // the rest of the search over the compacted window only
+        const uint32_t above = s;
+        uint32_t cw[kCandCap / 32];
+        const int wcnt = mid;
+#pragma unroll
+        for (int k = 0; k < kCandCap / 32; ++k) {
+          const int at = 32 * k + lane;
+          cw[k] = at < wcnt ? cand_all[warp][at] : 0u;  // 0 is below every candidate
         }
-        digit = __shfl_sync(kFull, digit, src);
-        above_new = __shfl_sync(kFull, above_new, src);
-        prefix |= unsigned(digit) << shift;
-        pmask |= 255u << shift;
-        above = above_new;
-        __syncwarp();
+#pragma unroll 1
+        for (; b >= 0; --b) {
+          const uint32_t t = x | (1u << b);
+          if (above + mass_at_least<kCandCap / 32>(cw, t) >= tgt) x = t;
+        }
+        tau = x;
+        keep_ties = (tgt - above - mass_at_least<kCandCap / 32>(cw, tau + 1) + tau - 1) / tau;
+        break;
+      } else if (stage == kBits) {
+        if (s >= tgt) x = c;
+        --b;
+      } else {  // kTies: s = G(tau + 1)
+        keep_ties = (tgt - s + tau - 1) / tau;
+        break;
       }
-      if (!keep_all) {
-        tau = prefix;
-        const unsigned long long mt = mass_fx(__uint_as_float(tau));  // > 0
-        keep_ties = (tgt - above + mt - 1) / mt;
+      // the next threshold
+      if (stage == kLead) {
+        if (lo < hi) {
+          mid = (lo + hi + 1) >> 1;
+          c = 1u << mid;
+          continue;
+        }
+        x = 1u << lo;
+        b = lo - 1;
+        int wcnt = 0;  // compact the window [x, 2x); order does not matter for sums
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+          const bool in = (m[i] - x) < x;  // unsigned: x <= m < 2x
+          const unsigned bal = __ballot_sync(kFull, in);
+          const int at = wcnt + __popc(bal & lanemask_lt());
+          if (in && at < kCandCap) cand_all[warp][at] = m[i];
+          wcnt += __popc(bal);
+        }
+        __syncwarp();
+        if (wcnt <= kCandCap) {
+          mid = wcnt;
+          c = x << 1;
+          stage = kAbove;
+          continue;
+        }
+        stage = kBits;
+      }
+      if (stage == kBits) {
+        if (b >= 0) {
+          c = x | (1u << b);
+          continue;
+        }
+        tau = x;
+        c = tau + 1u;
+        stage = kTies;
       }
     }
+  }
 
-    // ---- 4. STA union + compaction
-    int tq, hq, wq;
-    block_coords(g, blk, tq, hq, wq);
-    int32_t* out_idx = a.idx + (size_t(bh) * nb + blk) * nb;
-    int pos = 0;
-    unsigned long long ties = 0;
-    for (int base = 0; base < nb; base += 32) {
-      const int j = base + lane;
-      const bool valid = j < nb;
-      bool nab = false, tie = false;
-      if (valid) {
-        if (keep_all) {
-          nab = true;
-        } else {
-          const unsigned key = __float_as_uint(Lr[j]);
-          nab = key > tau;
-          tie = key == tau;
-        }
-      }
+  // ---- keep bitmap in shared memory: the NABLA bits by ballot (ties in
+  // index order), then OR the STA box, clipped to the grid
+  uint32_t* rbits = rbits_all[warp];
+  uint32_t ties = 0;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    if (32 * i < nb) {  // warp-uniform
+      const bool valid = lane + 32 * i < nb;
+      bool nab = valid && (keep_all || m[i] > tau);
+      const bool tie = valid && !keep_all && m[i] == tau;
       const unsigned tb = __ballot_sync(kFull, tie);
       if (tie) nab = (ties + __popc(tb & lanemask_lt())) < keep_ties;
       ties += __popc(tb);
-      bool in_sta = false;
-      if (valid && a.sta_t >= 0) {
-        int tk, hk, wk;
-        block_coords(g, j, tk, hk, wk);
-        in_sta = abs(tk - tq) <= a.sta_t && abs(hk - hq) <= a.sta_h && abs(wk - wq) <= a.sta_w;
-      }
-      const bool kept = valid && (nab || in_sta);
-      const unsigned kb = __ballot_sync(kFull, kept);
-      if (kept) out_idx[pos + __popc(kb & lanemask_lt())] = j;
-      pos += __popc(kb);
-      if (lane == 0) my_bits[base >> 5] = kb;
+      const unsigned kb = __ballot_sync(kFull, nab);
+      if (lane == 0) rbits[i] = kb;
     }
-    if (lane == 0) a.cnt[size_t(bh) * nb + blk] = pos;
-  } else {
-    for (int i = lane; i < nwords; i += 32) my_bits[i] = 0u;
   }
-  __syncthreads();
+  __syncwarp();
+  if (a.sta_t >= 0) {
+    int tq, hq, wq;
+    block_coords(g, qb, tq, hq, wq);
+    const int t0 = max(tq - a.sta_t, 0), t1 = min(tq + a.sta_t, g.T - 1);
+    const int h0 = max(hq - a.sta_h, 0), h1 = min(hq + a.sta_h, g.nh - 1);
+    const int w0 = max(wq - a.sta_w, 0), w1 = min(wq + a.sta_w, g.nw - 1);
+    const int nw_ = w1 - w0 + 1, nhw = (h1 - h0 + 1) * nw_;
+    const int cells = (t1 - t0 + 1) * nhw;
+    for (int cidx = lane; cidx < cells; cidx += 32) {
+      const int ct = cidx / nhw, r = cidx - ct * nhw, ch = r / nw_, cw = r - ch * nw_;
+      const int j = ((t0 + ct) * g.nh + h0 + ch) * g.nw + w0 + cw;
+      atomicOr(&rbits[j >> 5], 1u << (j & 31));
+    }
+    __syncwarp();
+  }
 
-  // ---- 5. per-tile union lists, ordered for the attention kernel: first the
-  // steps that pair the same patch in frames t and t+1 (one two-frame TMA box
-  // each), then the remaining blocks in ascending order. The probability
-  // buffer L is free now and holds the pairing bitmaps.
-  if (warp < kMaskRows / 2) {
-    const int tile = tile0 + warp;
-    if (tile < g.ntile) {
-      const uint32_t* ba = bits + size_t(2 * warp) * nwords;
-      const uint32_t* bb = bits + size_t(2 * warp + 1) * nwords;
-      uint32_t* u = reinterpret_cast<uint32_t*>(L) + size_t(warp) * 3 * nwords;
-      uint32_t* first = u + nwords;
-      uint32_t* second = first + nwords;
-      for (int w = lane; w < nwords; w += 32) {
-        u[w] = ba[w] | bb[w];
-        first[w] = 0u;
-        second[w] = 0u;
-      }
-      __syncwarp();
-      // greedy along time, one patch per lane
-      const int pf = g.nh * g.nw;
-      for (int p = lane; p < pf; p += 32) {
-        bool pending = false;
-        for (int t = 0; t < g.T; ++t) {
-          const int b = t * pf + p;
-          const bool in = (u[b >> 5] >> (b & 31)) & 1u;
-          if (pending && in) {
-            const int f = b - pf;
-            atomicOr(&first[f >> 5], 1u << (f & 31));
-            atomicOr(&second[b >> 5], 1u << (b & 31));
-            pending = false;
-          } else {
-            pending = in;
-          }
-        }
-      }
-      __syncwarp();
-      int32_t* out = a.tidx + (size_t(bh) * g.ntile + tile) * nb;
-      auto flags = [&](int b) {
-        return int(((ba[b >> 5] >> (b & 31)) & 1u) << 16) | int(((bb[b >> 5] >> (b & 31)) & 1u) << 17);
-      };
-      int pos = 0;
-      for (int w = 0; w < nwords; ++w) {
-        const uint32_t x = first[w];
-        if ((x >> lane) & 1u) {
-          const int b = w * 32 + lane;
-          const int o = pos + 2 * __popc(x & lanemask_lt());
-          out[o] = b | flags(b) | kEntryTPair;
-          out[o + 1] = (b + pf) | flags(b + pf);
-        }
-        pos += 2 * __popc(x);
-      }
-      for (int w = 0; w < nwords; ++w) {
-        const uint32_t x = u[w] & ~first[w] & ~second[w];
-        if ((x >> lane) & 1u) {
-          const int b = w * 32 + lane;
-          out[pos + __popc(x & lanemask_lt())] = b | flags(b);
-        }
-        pos += __popc(x);
-      }
-      if (lane == 0) a.tcnt[size_t(bh) * g.ntile + tile] = pos;
+  // ---- ascending kept list, bitmap and count to global: lane per word
+  const int nwords = bitmap_words(g);
+  uint32_t* bits = a.bits + size_t(row) * nwords;
+  int32_t* out_idx = a.idx + size_t(row) * nb;
+  int pos = 0;
+  for (int base = 0; base < nwords; base += 32) {
+    const int wi = base + lane;
+    uint32_t w = wi < nwords ? rbits[wi] : 0u;
+    if (wi < nwords) bits[wi] = w;
+    const int cnt = __popc(w);
+    int inc = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(kFull, inc, o);
+      if (lane >= o) inc += t;
     }
+    int o = pos + inc - cnt;
+    while (w) {
+      out_idx[o++] = 32 * wi + __ffs(w) - 1;
+      w &= w - 1u;
+    }
+    pos += __shfl_sync(kFull, inc, 31);
   }
+  if (lane == 0) a.cnt[row] = pos;
 }
 
-cudaError_t launch_mask(const MaskArgs& a, const Geometry& g, cudaStream_t stream) {
-  const size_t smem = mask_smem_bytes(g);
-  const dim3 grid(unsigned((g.ntile + kMaskRows / 2 - 1) / (kMaskRows / 2)), unsigned(g.BH));
-  cudaError_t e;
-  if (g.d == 128) {
-    e = cudaFuncSetAttribute(mask_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(smem));
-    if (e != cudaSuccess) return e;
-    mask_kernel<128><<<grid, kMaskThreads, smem, stream>>>(a, g);
-  } else {
-    e = cudaFuncSetAttribute(mask_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(smem));
-    if (e != cudaSuccess) return e;
-    mask_kernel<64><<<grid, kMaskThreads, smem, stream>>>(a, g);
+// ------------------------------------------------------------------ union
+constexpr int kUnionMaxWarps = 8;
+
+// Shared words per warp: the two rows' bitmaps (+1 zero word each, read by
+// the funnel shift below) and, frame-major ([T][fw] words, fw = words per
+// frame), the first blocks of the temporal pairs and the unpaired blocks.
+SA_HD int union_words_per_warp(const Geometry& g) {
+  const int fw = (g.nh * g.nw + 31) / 32;
+  return 2 * (bitmap_words(g) + 1) + 2 * g.T * fw;
+}
+
+__global__ void __launch_bounds__(kUnionMaxWarps * 32) union_kernel(MaskArgs a, Geometry g) {
+  extern __shared__ uint32_t ush[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwords = bitmap_words(g);
+  const int pf = g.nh * g.nw, fw = (pf + 31) >> 5, nf = g.T * fw;
+  const long item = long(blockIdx.x) * (blockDim.x >> 5) + warp;  // (bh, tile)
+  if (item >= long(g.BH) * g.ntile) return;
+  const int bh = int(item / g.ntile), tile = int(item - long(bh) * g.ntile);
+  int qa, qb;
+  tile_blocks(g, tile, qa, qb);
+  const uint32_t* ba = a.bits + (size_t(bh) * g.nb + qa) * nwords;
+  const uint32_t* bb = qb >= 0 ? a.bits + (size_t(bh) * g.nb + qb) * nwords : nullptr;
+  uint32_t* ua = ush + size_t(warp) * union_words_per_warp(g);
+  uint32_t* ub = ua + nwords + 1;
+  uint32_t* firstF = ub + nwords + 1;
+  uint32_t* leftF = firstF + nf;
+  for (int w = lane; w <= nwords; w += 32) {
+    ua[w] = w < nwords ? ba[w] : 0u;
+    ub[w] = (bb != nullptr && w < nwords) ? bb[w] : 0u;
   }
+  __syncwarp();
+
+  // Bits [t * pf + 32 w, +32) of the union, clipped to frame t.
+  auto frame_word = [&](int t, int w) -> uint32_t {
+    const int s = t * pf + 32 * w;
+    const int q = s >> 5, off = s & 31;
+    uint32_t x = ua[q] | ub[q];
+    if (off) x = (x >> off) | ((ua[q + 1] | ub[q + 1]) << (32 - off));
+    const int nbits = pf - 32 * w;
+    return nbits < 32 ? x & ((1u << nbits) - 1u) : x;
+  };
+  // Greedy pairing along time, 32 patches per lane-word at once: a block
+  // present in frame t whose frame t - 1 block is present and not already the
+  // second of a pair becomes the second of a pair.
+  for (int w = lane; w < fw; w += 32) {
+    uint32_t prev_in = 0u, prev_pair = 0u;
+    for (int t = 0; t < g.T; ++t) {
+      const uint32_t in = frame_word(t, w);
+      const uint32_t pair = prev_in & ~prev_pair & in;
+      if (t > 0) {
+        firstF[(t - 1) * fw + w] = pair;
+        leftF[(t - 1) * fw + w] = prev_in & ~prev_pair & ~pair;
+      }
+      prev_in = in;
+      prev_pair = pair;
+    }
+    firstF[(g.T - 1) * fw + w] = 0u;
+    leftF[(g.T - 1) * fw + w] = prev_in & ~prev_pair;
+  }
+  __syncwarp();
+
+  // Emission in ascending block order (frame-major words are in block
+  // order): first the pairs, two entries each, then the unpaired blocks.
+  // Each lane takes one word of a 32-word group; a warp scan places it.
+  int32_t* out = a.tidx + size_t(item) * g.nb;
+  auto flags = [&](int b) {
+    return int(((ua[b >> 5] >> (b & 31)) & 1u) << 16) | int(((ub[b >> 5] >> (b & 31)) & 1u) << 17);
+  };
+  int pos = 0;
+  for (int pass = 0; pass < 2; ++pass) {
+    const uint32_t* src = pass == 0 ? firstF : leftF;
+    for (int base = 0; base < nf; base += 32) {
+      const int it = base + lane;
+      uint32_t x = it < nf ? src[it] : 0u;
+      const int c = (pass == 0 ? 2 : 1) * __popc(x);
+      int inc = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(kFull, inc, o);
+        if (lane >= o) inc += v;
+      }
+      int o = pos + inc - c;
+      const int t = it / fw;
+      const int b0 = t * pf + 32 * (it - t * fw);
+      while (x) {
+        const int b = b0 + __ffs(x) - 1;
+        x &= x - 1u;
+        if (pass == 0) {
+          out[o] = b | flags(b) | kEntryTPair;
+          out[o + 1] = (b + pf) | flags(b + pf);
+          o += 2;
+        } else {
+          out[o++] = b | flags(b);
+        }
+      }
+      pos += __shfl_sync(kFull, inc, 31);
+    }
+  }
+  if (lane == 0) a.tcnt[item] = pos;
+}
+
+template <int VPL>
+cudaError_t launch_select(const MaskArgs& a, const Geometry& g, int ld, cudaStream_t stream) {
+  const long rows = long(g.BH) * g.nb;
+  select_kernel<VPL><<<unsigned((rows + kSelWarps - 1) / kSelWarps), kSelWarps * 32, 0, stream>>>(
+      a.logits, a, g, ld);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_logits(const MaskArgs& a, const Geometry& g, int ld, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(logits_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(kLogitSmem));
+  if (e != cudaSuccess) return e;
+  const dim3 grid(unsigned(ld / kBN), unsigned((g.nb + kBM - 1) / kBM), unsigned(g.BH));
+  logits_kernel<D><<<grid, kLogitThreads, kLogitSmem, stream>>>(a.qbar, a.kbar, a.logits, g, ld,
+                                                                a.scale);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_mask(const MaskArgs& a, const Geometry& g, cudaStream_t stream) {
+  const int ld = logits_ld(g);
+  cudaError_t e = g.d == 128 ? launch_logits<128>(a, g, ld, stream)
+                             : launch_logits<64>(a, g, ld, stream);
+  if (e != cudaSuccess) return e;
+  const int vpl = (g.nb + 31) / 32;  // nb <= 3072 (checked by the entry points)
+  if (vpl <= 4) e = launch_select<4>(a, g, ld, stream);
+  else if (vpl <= 8) e = launch_select<8>(a, g, ld, stream);
+  else if (vpl <= 16) e = launch_select<16>(a, g, ld, stream);
+  else if (vpl <= 32) e = launch_select<32>(a, g, ld, stream);
+  else if (vpl <= 64) e = launch_select<64>(a, g, ld, stream);
+  else e = launch_select<96>(a, g, ld, stream);
+  if (e != cudaSuccess) return e;
+  const long items = long(g.BH) * g.ntile;
+  const size_t warp_bytes = size_t(union_words_per_warp(g)) * sizeof(uint32_t);
+  int wpc = int((48 * 1024) / warp_bytes);  // warps per CTA within 48 KB
+  wpc = wpc < 1 ? 1 : (wpc > kUnionMaxWarps ? kUnionMaxWarps : wpc);
+  union_kernel<<<unsigned((items + wpc - 1) / wpc), unsigned(wpc * 32), wpc * warp_bytes,
+                 stream>>>(a, g);
   return cudaGetLastError();
 }
 
@@ -355,10 +540,10 @@ __global__ void __launch_bounds__(1024) tile_order_kernel(const int32_t* __restr
         const int partner = i ^ stride;
         if (partner > i) {
           const bool up = (i & size) == 0;
-          const uint32_t a = key[i], b = key[partner];
-          if ((a > b) == up) {
-            key[i] = b;
-            key[partner] = a;
+          const uint32_t x = key[i], y = key[partner];
+          if ((x > y) == up) {
+            key[i] = y;
+            key[partner] = x;
           }
         }
       }

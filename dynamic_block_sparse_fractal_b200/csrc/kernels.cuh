@@ -16,24 +16,25 @@ cudaError_t launch_pool(const void* q, const void* k, float* qbar, float* kbar, 
 cudaError_t launch_permute(const void* x, void* y, const Geometry& g, int inverse,
                            cudaStream_t stream);
 
-// Reduced map + CDF threshold + STA union -> per-q-block lists and per-tile
-// union lists. target_fx = round((1 - thr) * 2^40) (mass threshold in the
-// kernel's fixed point); dense = (thr == 0).
+// Reduced map + CDF threshold + STA union -> per-q-block lists and keep
+// bitmaps, then per-tile union lists. target_fx = round((1 - thr) * 2^30)
+// (mass threshold in the select kernel's fixed point); dense = (thr == 0).
 struct MaskArgs {
   const float* qbar;
   const float* kbar;
+  float* logits;   // [BH][nb][logits_ld(g)]
+  uint32_t* bits;  // [BH][nb][bitmap_words(g)]
   int32_t* cnt;
   int32_t* idx;
   int32_t* tcnt;
   int32_t* tidx;
-  uint32_t* status;
-  unsigned long long target_fx;
+  uint32_t target_fx;
   int dense;
   int sta_t, sta_h, sta_w;  // half-widths (window / 2), -1 = no STA
   float scale;              // 1 / sqrt(d)
 };
+// Three launches: logits GEMM, row select, tile union.
 cudaError_t launch_mask(const MaskArgs& a, const Geometry& g, cudaStream_t stream);
-size_t mask_smem_bytes(const Geometry& g);
 
 // Per head: tiles sorted by descending union length (ties by tile index).
 cudaError_t launch_tile_order(const int32_t* tcnt, int32_t* order, const Geometry& g,
