@@ -250,7 +250,7 @@ def run_ours(args, w, rank, world):
                 "ms_per_step": round(e2e_ms, 3),
                 "h2d_bytes_per_step": int(3 * q.numel() * 2),
                 "d2h_bytes_per_step": int(out.numel() * out.element_size())},
-        "gpu_launches": 4 * args.steps,  # pool, mask, tile order, attention
+        "gpu_launches": 6 * args.steps,  # pool, logits, select, union, tile order, attention
         "clocks": clocks.summary(),
     }
     if dist is not None:

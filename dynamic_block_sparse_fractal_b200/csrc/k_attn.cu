@@ -55,8 +55,9 @@ constexpr int kChunkBytes = 128 * 128;  // 128 rows x 128 B (64 bf16 channels)
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Column pairs (of every 8) whose exp2 runs on the FMA pipe instead of the
-// SFU. Measured on the HunyuanVideo-like workload: the SFU is not yet the
-// limit, and 3 of 8 made the softmax 1.7x slower, so all go to the SFU.
+// SFU. Measured on the HunyuanVideo-like workload: 1 of 8 made the attention
+// 7% slower and 2 of 8 17% slower (the softmax warps are limited by issue and
+// latency, not by the SFU's rate), so all go to the SFU.
 constexpr int kPolyPairsPer8 = 0;
 constexpr int kMaxList = 2880;             // largest union: nb <= 2880 blocks
 
@@ -71,7 +72,6 @@ struct __align__(1024) AttnSmem {
   uint64_t q_full[2];
   uint64_t full[kSlots];
   uint64_t empty[kSlots];
-  uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t o_final[2];
   uint64_t drain;
@@ -129,6 +129,18 @@ __device__ __forceinline__ void fail(uint32_t* status, int* abort, uint32_t bit)
   *reinterpret_cast<volatile int*>(abort) = 1;
 }
 
+// Ring position of S_X(step) in the MMA issue order
+//   S_A0 S_B0 | PV_A(j) S_A(j+1) PV_B(j) S_B(j+1) | ...
+// (n0, n1 = the tiles' step counts). The commit that frees this K slot is
+// also the softmax's signal that S_X(step) is complete.
+__device__ __forceinline__ int s_op_index(int x, int step, int n0, int n1) {
+  if (step == 0) return x == 0 ? 0 : (n0 > 0 ? 1 : 0);
+  const int i = step - 1;  // the loop iteration that issues S_X(step)
+  const int c = min(i, n0) + min(i, max(n0 - 1, 0)) + min(i, n1) + min(i, max(n1 - 1, 0));
+  const int base = (n0 > 0) + (n1 > 0) + c;
+  return x == 0 ? base + 1 : base + (i < n0) + (i + 1 < n0) + 1;
+}
+
 __device__ __forceinline__ int step_blocks(const Tile& t, int step) {
   return (t.n_u - 2 * step) >= 2 ? 2 : 1;
 }
@@ -169,7 +181,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm.abort = 0;
     for (int x = 0; x < 2; ++x) {
       mbar_init(&sm.q_full[x], 1);
-      mbar_init(&sm.s_full[x], 1);
       mbar_init(&sm.p_full[x], 128);
       mbar_init(&sm.o_final[x], 1);
     }
@@ -297,9 +308,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = mbar_wait(&sm.q_full[0], 0, abort);
       if (ok && n1 > 0) ok = mbar_wait(&sm.q_full[1], 0, abort);
       int k = 0;  // op index (ring position)
-      auto issue_s = [&](int x, int step) {
-        const int s = k & (kSlots - 1);
-        if (!mbar_wait(&sm.full[s], (k / kSlots) & 1, abort)) return false;
+      // S_X(step) = Q_X K^T into tile X's S columns, the K pair in slot s
+      auto mma_s = [&](int x, int step, int s) {
         const uint64_t qd = x ? qdesc1 : qdesc0;
         const uint64_t kd = kdesc0 + uint64_t(s) * kSlotStep;
         const uint32_t id = ((x ? u1 : u0) - 2 * step) >= 2 ? id_s2 : id_s1;
@@ -309,48 +319,68 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t off = (uint32_t(kk >> 2) * kChunkBytes + uint32_t(kk & 3) * 32u) >> 4;
           mma_ss(d_tmem, qd + off, kd + off, id, kk > 0);
         }
-        mma_commit(&sm.empty[s]);
-        mma_commit(&sm.s_full[x]);
-        ++k;
-        return true;
       };
-      auto issue_pv = [&](int x, int step) {
-        const int s = k & (kSlots - 1);
-        if (!mbar_wait(&sm.p_full[x], step & 1, abort)) return false;
-        if (!mbar_wait(&sm.full[s], (k / kSlots) & 1, abort)) return false;
-        tc_fence_after_sync();  // P was written by the softmax threads
+      // O_X += P_X V, P from tile X's S columns in TMEM, the V pair in slot s
+      auto mma_pv = [&](int x, int step, int s) {
         const uint64_t vd = vdesc0 + uint64_t(s) * kSlotStep;
         const uint32_t o_tmem = tmem + col_o(x);
         const uint32_t p_tmem = tmem + col_s(x);
-        const uint32_t acc0 = step > 0 ? 1u : 0u;
+        mma_ts(o_tmem, p_tmem, vd, id_pv, step > 0 ? 1u : 0u);
         if (((x ? u1 : u0) - 2 * step) >= 2) {
-          mma_ts(o_tmem, p_tmem, vd, id_pv, acc0);
 #pragma unroll
           for (int kk = 1; kk < 8; ++kk)
             mma_ts(o_tmem, p_tmem + uint32_t(kk) * 8u, vd + uint32_t(kk) * 128u, id_pv, 1u);
         } else {
-          mma_ts(o_tmem, p_tmem, vd, id_pv, acc0);
 #pragma unroll
           for (int kk = 1; kk < 4; ++kk)
             mma_ts(o_tmem, p_tmem + uint32_t(kk) * 8u, vd + uint32_t(kk) * 128u, id_pv, 1u);
         }
-        mma_commit(&sm.empty[s]);
-        if (step == (x ? n1 : n0) - 1) mma_commit(&sm.o_final[x]);
-        ++k;
-        return true;
       };
-      // the order OpIter describes: S_A0 S_B0 | PV_A(j) S_A(j+1) PV_B(j) S_B(j+1) | ...
-      if (ok && n0 > 0) ok = issue_s(0, 0);
-      if (ok && n1 > 0) ok = issue_s(1, 0);
+      // the order the producers fill: S_A0 S_B0 | PV_A(j) S_A(j+1) PV_B(j) S_B(j+1) | ...
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        if (!ok || (x ? n1 : n0) == 0) continue;
+        const int s = k & (kSlots - 1);
+        ok = mbar_wait(&sm.full[s], (k / kSlots) & 1, abort);
+        if (!ok) break;
+        mma_s(x, 0, s);
+        mma_commit(&sm.empty[s]);  // also tells the softmax that S_X(0) is complete
+        ++k;
+      }
+      // One unit per tile and step: PV_X(j) and S_X(j+1) issued back to back
+      // behind one round of waits (an idle tensor core between the two would
+      // cost more than waiting for the K pair a little earlier).
       const int nmax = n0 > n1 ? n0 : n1;
       for (int j = 0; ok && j < nmax; ++j) {
-        if (j < n0) {
-          ok = issue_pv(0, j);
-          if (ok && j + 1 < n0) ok = issue_s(0, j + 1);
-        }
-        if (ok && j < n1) {
-          ok = issue_pv(1, j);
-          if (ok && j + 1 < n1) ok = issue_s(1, j + 1);
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          const int nx = x ? n1 : n0;
+          if (!ok || j >= nx) continue;
+          const bool has_s = j + 1 < nx;
+          const int s_pv = k & (kSlots - 1), s_s = (k + 1) & (kSlots - 1);
+          const uint32_t par_pv = (k / kSlots) & 1, par_s = ((k + 1) / kSlots) & 1;
+          // one round trip for all three barriers; a bounded wait only for
+          // those not yet complete
+          const uint32_t ready = mbar_peek3(&sm.p_full[x], j & 1, &sm.full[s_pv], par_pv,
+                                            has_s ? &sm.full[s_s] : &sm.full[s_pv],
+                                            has_s ? par_s : par_pv);
+          if (ready != 7u) {
+            ok = ((ready & 1u) || mbar_wait(&sm.p_full[x], j & 1, abort)) &&
+                 ((ready & 2u) || mbar_wait(&sm.full[s_pv], par_pv, abort)) &&
+                 ((ready & 4u) || !has_s || mbar_wait(&sm.full[s_s], par_s, abort));
+            if (!ok) break;
+          }
+          tc_fence_after_sync();  // P was written by the softmax threads
+          mma_pv(x, j, s_pv);
+          mma_commit(&sm.empty[s_pv]);
+          if (has_s) {
+            mma_s(x, j + 1, s_s);
+            mma_commit(&sm.empty[s_s]);  // also tells the softmax that S_X(j+1) is complete
+            k += 2;
+          } else {
+            mma_commit(&sm.o_final[x]);
+            k += 1;
+          }
         }
       }
       if (!ok) {
@@ -383,7 +413,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int e1 = nblk == 2 ? t.list[2 * j + 1] : 0;
       const bool keep0 = row_valid && (e0 & keep_bit);
       const bool keep1 = row_valid && nblk == 2 && (e1 & keep_bit);
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sm.s_full[x], j & 1, abort));
+      const int ks = s_op_index(x, j, tile[0].nsteps, tile[1].nsteps);
+      ok = __all_sync(0xFFFFFFFFu,
+                      mbar_wait(&sm.empty[ks & (kSlots - 1)], (ks / kSlots) & 1, abort));
       if (!ok) break;
       tc_fence_after_sync();
       // keep0 / keep1 are uniform across a warp (a warp's rows lie in one
@@ -398,17 +430,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
       }
       tmem_wait_ld();
-      float mx = -INFINITY;
+      // row max over four independent chains (a single chain of 64 dependent
+      // max3 would cost its full latency)
+      float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (keep0) {
 #pragma unroll
         for (int i = 0; i < 64; i += 2)
-          mx = max3(mx, __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
+          mq[(i >> 1) & 3] = max3(mq[(i >> 1) & 3], __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
       }
       if (keep1) {
 #pragma unroll
         for (int i = 64; i < 128; i += 2)
-          mx = max3(mx, __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
+          mq[(i >> 1) & 3] = max3(mq[(i >> 1) & 3], __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
       }
+      float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
       mx *= sl2;
       const bool need = mx > m + kRescaleThreshold;  // false while mx = -inf
       const float m_new = need ? mx : m;
@@ -431,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // kPolyPairsPer8 of every 8 column pairs take the FMA-pipe exp2.
       const uint64_t sl2x2 = f2_pack(sl2, sl2);
       const uint64_t negm2 = f2_pack(-m, -m);
-      uint64_t rs2 = f2_pack(0.f, 0.f);
+      uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};  // four independent packed sums
 #pragma unroll
       for (int i = 0; i < 64; ++i) {
         const bool kp = (2 * i) < 64 ? keep0 : keep1;
@@ -448,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             e2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
           }
-          rs2 = f2_add(rs2, e2);
+          rs2[i & 3] = f2_add(rs2[i & 3], e2);
           float p0, p1;
           f2_unpack(e2, p0, p1);
           packed = pack_bf16x2(p0, p1);
@@ -456,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         sv[i] = packed;
       }
       float rs_lo, rs_hi;
-      f2_unpack(rs2, rs_lo, rs_hi);
+      f2_unpack(f2_add(f2_add(rs2[0], rs2[1]), f2_add(rs2[2], rs2[3])), rs_lo, rs_hi);
       const float rs = rs_lo + rs_hi;
       l += rs;
       tmem_st32(s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
