@@ -189,29 +189,52 @@ def run_ours(args, w, rank, world):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms = float(t.item())
 
-    # ---- end to end through the public API, host buffers, copies timed
+    # ---- end to end through the public API, host buffers, copies timed.
+    # Every step copies its Q/K/V from pinned host memory and its output back;
+    # as a serving loop would, consecutive steps are double-buffered on three
+    # streams (step i+1's inputs travel while step i computes, step i's output
+    # travels while step i+1 computes).
     pin = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).reshape(w.B, w.H, w.S, w.d)
            .pin_memory() for x in (q_h, k_h, v_h)]
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    e2e_steps = max(1, min(args.steps, 5))
+    out_h = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    e2e_steps = max(2, min(args.steps, 10))
     attn = api.NablaAttention(w.B, w.H, w.T, w.Hh, w.Ww, w.d, w.thr, w.sta, device=dev)
+    s_h2d, s_cmp, s_d2h = (torch.cuda.Stream(dev) for _ in range(3))
+    bufs = [[torch.empty_like(q) for _ in range(3)] for _ in range(2)]
+    outs = [torch.empty_like(out) for _ in range(2)]
+    ev_in = [torch.cuda.Event() for _ in range(2)]    # inputs of buffer b landed
+    ev_done = [torch.cuda.Event() for _ in range(2)]  # compute on buffer b finished
+    ev_out = [torch.cuda.Event() for _ in range(2)]   # output of buffer b copied back
 
-    def e2e_step():
-        qd = pin[0].to(dev, non_blocking=True)
-        kd = pin[1].to(dev, non_blocking=True)
-        vd = pin[2].to(dev, non_blocking=True)
-        o = attn(qd, kd, vd)
-        out_h.copy_(o, non_blocking=True)
+    def e2e_step(i):
+        b = i & 1
+        with torch.cuda.stream(s_h2d):
+            if i >= 2:
+                s_h2d.wait_event(ev_done[b])  # the previous user of buffer b read its inputs
+            for dst, src in zip(bufs[b], pin):
+                dst.copy_(src, non_blocking=True)
+            ev_in[b].record(s_h2d)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(ev_in[b])
+            if i >= 2:
+                s_cmp.wait_event(ev_out[b])  # outs[b] was copied back
+            attn(bufs[b][0], bufs[b][1], bufs[b][2], out=outs[b], stream=s_cmp)
+            ev_done[b].record(s_cmp)
+        with torch.cuda.stream(s_d2h):
+            s_d2h.wait_event(ev_done[b])
+            out_h[b].copy_(outs[b], non_blocking=True)
+            ev_out[b].record(s_d2h)
 
-    e2e_step()
+    e2e_step(0)
+    e2e_step(1)
     torch.cuda.synchronize(dev)
     barrier()
     a0 = torch.cuda.Event(enable_timing=True)
     a1 = torch.cuda.Event(enable_timing=True)
-    a0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    a1.record(stream)
+    a0.record(s_h2d)
+    for i in range(2, 2 + e2e_steps):
+        e2e_step(i)
+    a1.record(s_d2h)
     torch.cuda.synchronize(dev)
     barrier()
     e2e_ms = a0.elapsed_time(a1) / e2e_steps
@@ -219,7 +242,7 @@ def run_ours(args, w, rank, world):
         t = torch.tensor([e2e_ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_ms = float(t.item())
-    st = attn.check()
+    st = attn.check(s_cmp)
     if st != api.SA_OK:
         raise SystemExit(f"device status after e2e: {api.status_string(st)}")
 
@@ -247,7 +270,8 @@ def run_ours(args, w, rank, world):
                      "traffic": None, "kernel": "sa::attn_kernel<128>",
                      "peak_source": f"{src} bf16 burst"},
         "e2e": {"value": round(world * kept_flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
-                "ms_per_step": round(e2e_ms, 3),
+                "ms_per_step": round(e2e_ms, 3), "steps": e2e_steps,
+                "overlap": "double-buffered: H2D of step i+1 and D2H of step i-1 overlap step i",
                 "h2d_bytes_per_step": int(3 * q.numel() * 2),
                 "d2h_bytes_per_step": int(out.numel() * out.element_size())},
         "gpu_launches": 6 * args.steps,  # pool, logits, select, union, tile order, attention
@@ -327,10 +351,16 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="run the workload's grid with this many heads (small ncu captures); "
+                         "the line's config then names the changed workload")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     w = pick_workload(args.workload)
+    if args.heads is not None:
+        import dataclasses
+        w = dataclasses.replace(w, H=args.heads, name=f"{w.name}_heads{args.heads}")
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", str(args.gpus if args.gpus == 1 else 1)))
     if args.impl == "reference":
