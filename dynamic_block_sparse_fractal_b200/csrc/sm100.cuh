@@ -187,6 +187,73 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 
+// Eight back-to-back MMAs over K = 8 x 16 in one asm block (no compiler
+// instructions between them): D[tmem] (+)= A * B^T with A and B both
+// 128-byte-swizzled K-major shared-memory tiles whose 64-element K chunks are
+// kChunk bytes apart. Descriptors are passed as 32-bit halves; the per-MMA
+// offsets move only the start-address field (low word, no carry). The first
+// MMA accumulates iff acc != 0, the other seven always do.
+template <uint32_t kChunk>
+__device__ __forceinline__ void mma_ss_k8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t acc) {
+  const uint32_t alo = uint32_t(a_desc), ahi = uint32_t(a_desc >> 32);
+  const uint32_t blo = uint32_t(b_desc), bhi = uint32_t(b_desc >> 32);
+#define SA_MMA_SS_STEP(KK, PRED)                                                     \
+  "add.u32 la, %1, " #KK ";\n\t"                                                   \
+  "add.u32 lb, %3, " #KK ";\n\t"                                                   \
+  "mov.b64 da, {la, %2};\n\t"                                                      \
+  "mov.b64 db, {lb, %4};\n\t"                                                      \
+  "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, " PRED ";\n\t"
+  asm volatile(
+      "{\n\t.reg .pred p0, p1;\n\t.reg .u32 la, lb;\n\t.reg .b64 da, db;\n\t"
+      "setp.ne.b32 p0, %6, 0;\n\t"
+      "setp.eq.b32 p1, 0, 0;\n\t"
+      SA_MMA_SS_STEP(%7, "p0") SA_MMA_SS_STEP(%8, "p1") SA_MMA_SS_STEP(%9, "p1")
+      SA_MMA_SS_STEP(%10, "p1") SA_MMA_SS_STEP(%11, "p1") SA_MMA_SS_STEP(%12, "p1")
+      SA_MMA_SS_STEP(%13, "p1") SA_MMA_SS_STEP(%14, "p1") "}"
+      ::"r"(d_tmem), "r"(alo), "r"(ahi), "r"(blo), "r"(bhi), "r"(idesc), "r"(acc),
+      "n"(0), "n"(2), "n"(4), "n"(6), "n"(kChunk / 16), "n"(kChunk / 16 + 2),
+      "n"(kChunk / 16 + 4), "n"(kChunk / 16 + 6)
+      : "memory");
+#undef SA_MMA_SS_STEP
+}
+
+// NK (4 or 8) back-to-back MMAs with A from TMEM (8 columns of bf16 pairs per
+// K step of 16) and B an MN-major shared-memory tile advancing 2048 bytes per
+// K step; the first accumulates iff acc != 0, the others always do.
+template <int NK>
+__device__ __forceinline__ void mma_ts_k(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t acc) {
+  static_assert(NK == 4 || NK == 8, "NK is 4 or 8");
+  const uint32_t blo = uint32_t(b_desc), bhi = uint32_t(b_desc >> 32);
+#define SA_MMA_TS_STEP(TOFF, BOFF, PRED)                                             \
+  "add.u32 ta, %1, " #TOFF ";\n\t"                                                  \
+  "add.u32 lb, %2, " #BOFF ";\n\t"                                                  \
+  "mov.b64 db, {lb, %3};\n\t"                                                      \
+  "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %4, " PRED ";\n\t"
+  if constexpr (NK == 8) {
+    asm volatile(
+        "{\n\t.reg .pred p0, p1;\n\t.reg .b32 ta, lb;\n\t.reg .b64 db;\n\t"
+        "setp.ne.b32 p0, %5, 0;\n\t"
+        "setp.eq.b32 p1, 0, 0;\n\t"
+        SA_MMA_TS_STEP(0, 0, "p0") SA_MMA_TS_STEP(8, 128, "p1") SA_MMA_TS_STEP(16, 256, "p1")
+        SA_MMA_TS_STEP(24, 384, "p1") SA_MMA_TS_STEP(32, 512, "p1") SA_MMA_TS_STEP(40, 640, "p1")
+        SA_MMA_TS_STEP(48, 768, "p1") SA_MMA_TS_STEP(56, 896, "p1") "}"
+        ::"r"(d_tmem), "r"(a_tmem), "r"(blo), "r"(bhi), "r"(idesc), "r"(acc)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p0, p1;\n\t.reg .b32 ta, lb;\n\t.reg .b64 db;\n\t"
+        "setp.ne.b32 p0, %5, 0;\n\t"
+        "setp.eq.b32 p1, 0, 0;\n\t"
+        SA_MMA_TS_STEP(0, 0, "p0") SA_MMA_TS_STEP(8, 128, "p1") SA_MMA_TS_STEP(16, 256, "p1")
+        SA_MMA_TS_STEP(24, 384, "p1") "}"
+        ::"r"(d_tmem), "r"(a_tmem), "r"(blo), "r"(bhi), "r"(idesc), "r"(acc)
+        : "memory");
+  }
+#undef SA_MMA_TS_STEP
+}
+
 // Arrives once on *bar when every tensor-core op issued so far by this thread
 // has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
