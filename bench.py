@@ -64,6 +64,21 @@ def kept_flops_per_pair(w):
     return 4.0 * w.N * w.N * w.d
 
 
+def max_over_ranks(ms, dist, device):
+    """The slowest rank's time (every rank runs the same collective)."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tflops(world, flops_per_rank, ms):
+    """Whole-job throughput: every rank processes flops_per_rank in (the max) ms."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples during the timed region."""
 
@@ -184,10 +199,7 @@ def run_ours(args, w, rank, world):
     st = api.check(desc, ws)
     if st != api.SA_OK:
         raise SystemExit(f"device status after timing: {api.status_string(st)}")
-    if dist is not None:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dist, dev)
 
     # ---- end to end through the public API, host buffers, copies timed.
     # Every step copies its Q/K/V from pinned host memory and its output back;
@@ -238,10 +250,7 @@ def run_ours(args, w, rank, world):
     torch.cuda.synchronize(dev)
     barrier()
     e2e_ms = a0.elapsed_time(a1) / e2e_steps
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
     st = attn.check(s_cmp)
     if st != api.SA_OK:
         raise SystemExit(f"device status after e2e: {api.status_string(st)}")
@@ -252,7 +261,7 @@ def run_ours(args, w, rank, world):
     attn_tflops = kept_flops / (fwd_avg * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
     line = {
-        "metric": METRIC, "value": round(world * kept_flops / (ms_step * 1e-3) / 1e12, 2),
+        "metric": METRIC, "value": round(aggregate_tflops(world, kept_flops, ms_step), 2),
         "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -269,7 +278,7 @@ def run_ours(args, w, rank, world):
                      "unit": "TFLOP/s", "frac": round(attn_tflops / peak, 4),
                      "traffic": None, "kernel": "sa::attn_kernel<128>",
                      "peak_source": f"{src} bf16 burst"},
-        "e2e": {"value": round(world * kept_flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+        "e2e": {"value": round(aggregate_tflops(world, kept_flops, e2e_ms), 2), "unit": UNIT,
                 "ms_per_step": round(e2e_ms, 3), "steps": e2e_steps,
                 "overlap": "double-buffered: H2D of step i+1 and D2H of step i-1 overlap step i",
                 "h2d_bytes_per_step": int(3 * q.numel() * 2),
