@@ -64,6 +64,31 @@ def kept_flops_per_pair(w):
     return 4.0 * w.N * w.N * w.d
 
 
+# DRAM bytes (read + write) of one attention launch on the HunyuanVideo-like
+# workload, from the one-pass ncu capture in
+# profiles/launches_hunyuan_1x24x126720x128.md. Reported only while the
+# attention kernel's sources are the ones that capture measured.
+ATTN_TRAFFIC = {
+    "workload": "hunyuan_1x24x126720x128",
+    "bytes": 5.03e9 + 0.864e9,
+    "sources_sha1": "7dd48fe2c017a1bee8bc00062e38be73558fe3d1",
+}
+ATTN_SOURCES = ("k_attn.cu", "sm100.cuh", "exp2_poly.cuh", "layout.cuh", "kernels.cuh")
+
+
+def attn_traffic(w):
+    """Measured DRAM bytes per attention launch, or None if stale or another workload."""
+    import hashlib
+    if w.name != ATTN_TRAFFIC["workload"]:
+        return None
+    h = hashlib.sha1()
+    csrc = os.path.join(ROOT, "dynamic_block_sparse_fractal_b200", "csrc")
+    for f in ATTN_SOURCES:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return ATTN_TRAFFIC["bytes"] if h.hexdigest() == ATTN_TRAFFIC["sources_sha1"] else None
+
+
 def max_over_ranks(ms, dist, device):
     """The slowest rank's time (every rank runs the same collective)."""
     if dist is None:
@@ -276,7 +301,7 @@ def run_ours(args, w, rank, world):
         "computed_over_kept": round(computed_flops / kept_flops, 4),
         "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 2), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(attn_tflops / peak, 4),
-                     "traffic": None, "kernel": "sa::attn_kernel<128>",
+                     "traffic": attn_traffic(w), "kernel": "sa::attn_kernel<128>",
                      "peak_source": f"{src} bf16 burst"},
         "e2e": {"value": round(aggregate_tflops(world, kept_flops, e2e_ms), 2), "unit": UNIT,
                 "ms_per_step": round(e2e_ms, 3), "steps": e2e_steps,
