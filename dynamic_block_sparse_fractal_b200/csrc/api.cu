@@ -86,10 +86,21 @@ sa_status sparse_attn_plan(const sa_desc* desc, const void* q, const void* k, vo
 
   cudaError_t e = cudaMemsetAsync(at<uint32_t>(workspace, w.status), 0, 256, s);
   if (e != cudaSuccess) return SA_ERR_CUDA;
-  e = launch_pool(q, k, at<float>(workspace, w.qbar), at<float>(workspace, w.kbar), g, s);
+  e = launch_pool(q, k, at<float>(workspace, w.qbar), at<float>(workspace, w.kbar),
+                  at<float>(workspace, w.qsplit), at<float>(workspace, w.ksplit), g, s);
   if (e != cudaSuccess) return SA_ERR_CUDA;
 
   MaskArgs m;
+  std::memset(&m, 0, sizeof(m));
+  const long long rows = (long long)g.BH * g.nb;
+  const float* qsplit = at<float>(workspace, w.qsplit);
+  const float* ksplit = at<float>(workspace, w.ksplit);
+  if (!encode_rows_f32(&m.map_qhi, qsplit, rows, g.d, 128) ||
+      !encode_rows_f32(&m.map_qlo, qsplit + rows * g.d, rows, g.d, 128) ||
+      !encode_rows_f32(&m.map_khi, ksplit, rows, g.d, 256) ||
+      !encode_rows_f32(&m.map_klo, ksplit + rows * g.d, rows, g.d, 256))
+    return SA_ERR_CUDA;
+  m.status = at<uint32_t>(workspace, w.status);
   m.qbar = at<float>(workspace, w.qbar);
   m.kbar = at<float>(workspace, w.kbar);
   m.logits = at<float>(workspace, w.logits);

@@ -1,9 +1,10 @@
 // Mask build (NABLA, Metodologia 2 "Attenzione Ridotta" + "CDF Thresholding",
 // Metodologia 3 STA union), three kernels after the pooling:
 //
-//  logits_kernel  L[bh][r][j] = Qbar[r] . Kbar[j] / sqrt(d) for every pair of
-//                 blocks of a head in fp32 FFMA (register-tiled 128 x 128
-//                 output tiles), stored in the workspace;
+//  logits_tc_kernel  L[bh][r][j] = Qbar[r] . Kbar[j] / sqrt(d) for every pair
+//                 of blocks of a head on the TF32 tensor cores (three products
+//                 of a hi / lo split: fp32-level accuracy), 128 x 256 output
+//                 tiles, stored in the workspace;
 //  select_kernel  one warp per q-block row, the row held in registers:
 //                 softmax, then the CDF threshold without sorting. k-block j
 //                 is kept iff the probability mass ranked before it (descending
@@ -31,6 +32,11 @@ namespace {
 
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
+__device__ __forceinline__ void fail_status(uint32_t* status, int* abort, uint32_t bit) {
+  atomicOr(status, bit);
+  *reinterpret_cast<volatile int*>(abort) = 1;
+}
+
 __device__ __forceinline__ unsigned lanemask_lt() {
   unsigned m;
   asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
@@ -38,110 +44,153 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 }
 
 // ------------------------------------------------------------------ logits
-constexpr int kBM = 128, kBN = 128, kBK = 32, kPad = 4;
-constexpr int kLds = kBM + kPad;  // row pitch of a transposed slice (floats)
-constexpr int kLogitThreads = 256;
-constexpr size_t kLogitSmem = size_t(2) * 2 * kBK * kLds * sizeof(float);  // 67,584 B
+// L = Qbar Kbar^T / sqrt(d) per head on the TF32 tensor cores, in three
+// products of the pooled means' hi / lo split (hi*hi + hi*lo + lo*hi), fp32
+// accumulation in TMEM. One CTA per 128 x 256 output tile: warp 0 loads
+// 32-channel K-chunks of the four operands by TMA into a 2-stage ring, warp
+// 1 issues the MMAs (M=128, N=256, K=8), warps 2-5 read the accumulator,
+// scale it and store whole rows (staged through shared memory so the global
+// stores are coalesced).
+constexpr int kLtM = 128, kLtN = 256, kLtK = 32;  // tile rows, columns, K-chunk (128 B of fp32)
+constexpr int kLtThreads = 192;
+constexpr int kLtStagePitch = kLtN + 4;  // floats per staged output row (conflict-free)
+constexpr uint32_t kLtStageBytes = 2u * kLtM * kLtK * 4u + 2u * kLtN * kLtK * 4u;  // 96 KB
 
-// Rows [r0, r0 + 128) x channels [k0, k0 + 32) of a [nb][D] fp32 matrix,
-// 4 float4 per thread; rows past nb read as zeros.
+struct __align__(1024) LogitsSmem {
+  float a[2][2][kLtM * kLtK];  // [stage][hi, lo]: 128 rows x 128 B, 128-byte swizzle
+  float b[2][2][kLtN * kLtK];  // [stage][hi, lo]: 256 rows x 128 B
+  uint64_t full[2], empty[2], acc_full;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(4 * 32 * kLtStagePitch * 4 <= sizeof(float) * 2 * 2 * (kLtM + kLtN) * kLtK,
+              "the output staging reuses the operand stages");
+
 template <int D>
-__device__ __forceinline__ void load_slice(const float* __restrict__ m, int nb, int r0, int k0,
-                                           float4 (&v)[4]) {
-  const int t = threadIdx.x;
-#pragma unroll
-  for (int s = 0; s < 4; ++s) {
-    const int row = (t >> 3) + 32 * s;
-    v[s] = (r0 + row < nb)
-               ? __ldg(reinterpret_cast<const float4*>(m + size_t(r0 + row) * D + k0) + (t & 7))
-               : make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-}
-
-// Stores a slice transposed, dst[k][row] (channel-major, padded pitch).
-__device__ __forceinline__ void store_slice(float* dst, const float4 (&v)[4]) {
-  const int t = threadIdx.x;
-#pragma unroll
-  for (int s = 0; s < 4; ++s) {
-    const int row = (t >> 3) + 32 * s, k = 4 * (t & 7);
-    dst[(k + 0) * kLds + row] = v[s].x;
-    dst[(k + 1) * kLds + row] = v[s].y;
-    dst[(k + 2) * kLds + row] = v[s].z;
-    dst[(k + 3) * kLds + row] = v[s].w;
-  }
-}
-
-// CTA = one 128 x 128 tile of one head's nb x nb logits; thread (ty, tx)
-// accumulates 8 x 8 outputs: rows r0 + 8 ty + i, columns c0 + 4 tx + j and
-// c0 + 64 + 4 tx + j (two float4 groups, so that a quarter-warp's shared
-// loads hit distinct banks and its global stores are contiguous).
-// Channel slices of 32 are double-buffered: the next slice is fetched into
-// registers while the current one is multiplied out of shared memory.
-template <int D>
-__global__ void __launch_bounds__(kLogitThreads, 1)
-    logits_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
-                  float* __restrict__ L, Geometry g, int ld, float scale) {
-  extern __shared__ __align__(16) float lsm[];
-  float* As = lsm;                 // [2][kBK][kLds]
-  float* Bs = lsm + 2 * kBK * kLds;  // [2][kBK][kLds]
+__global__ void __launch_bounds__(kLtThreads, 1)
+    logits_tc_kernel(const __grid_constant__ MaskArgs a, Geometry g, int ld) {
+  extern __shared__ uint8_t lt_raw[];
+  LogitsSmem& sm = *reinterpret_cast<LogitsSmem*>(
+      (reinterpret_cast<uintptr_t>(lt_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int kChunks = D / kLtK;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.z;
-  const int r0 = blockIdx.y * kBM, c0 = blockIdx.x * kBN;
-  const float* qa = qbar + size_t(bh) * g.nb * D;
-  const float* kb = kbar + size_t(bh) * g.nb * D;
-  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
-  float acc[8][8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-
-  float4 ra[4], rb[4];
-  load_slice<D>(qa, g.nb, r0, 0, ra);
-  load_slice<D>(kb, g.nb, c0, 0, rb);
-  store_slice(As, ra);
-  store_slice(Bs, rb);
+  const int r0 = blockIdx.y * kLtM, c0 = blockIdx.x * kLtN;
+  const int row_base = bh * g.nb;  // first row of this head in the [BH*nb][d] operands
+  if (threadIdx.x == 0) {
+    sm.abort = 0;
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1);
+    }
+    mbar_init(&sm.acc_full, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
   __syncthreads();
-  constexpr int kSlices = D / kBK;
+  tc_fence_after_sync();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort = &sm.abort;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tensormap(&a.map_qhi);
+      prefetch_tensormap(&a.map_qlo);
+      prefetch_tensormap(&a.map_khi);
+      prefetch_tensormap(&a.map_klo);
+      int issued = -1;
+      for (int c = 0; c < kChunks; ++c) {
+        const int s = c & 1;
+        if (c >= 2 && !mbar_wait(&sm.empty[s], ((c >> 1) - 1) & 1, abort)) {
+          fail_status(a.status, &sm.abort, kDevErrTimeoutLoad);
+          break;
+        }
+        if (*abort) break;
+        mbar_arrive_expect_tx(&sm.full[s], kLtStageBytes);
+        tma_load_2d(sm.a[s][0], &a.map_qhi, &sm.full[s], c * kLtK, row_base + r0);
+        tma_load_2d(sm.a[s][1], &a.map_qlo, &sm.full[s], c * kLtK, row_base + r0);
+        tma_load_2d(sm.b[s][0], &a.map_khi, &sm.full[s], c * kLtK, row_base + c0);
+        tma_load_2d(sm.b[s][1], &a.map_klo, &sm.full[s], c * kLtK, row_base + c0);
+        issued = c;
+      }
+      if (*abort) {  // let this thread's copies land before the CTA can exit
+        int never = 0;
+        for (int c = issued; c >= 0 && c > issued - 2; --c)
+          mbar_wait(&sm.full[c & 1], (c >> 1) & 1, &never);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_tf32_f32(kLtM, kLtN);
+      bool ok = true;
+      for (int c = 0; c < kChunks && ok; ++c) {
+        const int s = c & 1;
+        ok = mbar_wait(&sm.full[s], (c >> 1) & 1, abort);
+        if (!ok) break;
+        tc_fence_after_sync();
+        const uint64_t ahi = sw128_desc(smem_u32(sm.a[s][0]), 16, 1024);
+        const uint64_t alo = sw128_desc(smem_u32(sm.a[s][1]), 16, 1024);
+        const uint64_t bhi = sw128_desc(smem_u32(sm.b[s][0]), 16, 1024);
+        const uint64_t blo = sw128_desc(smem_u32(sm.b[s][1]), 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < kLtK / 8; ++kk) {  // K = 8 tf32 = 32 B per MMA
+          const uint32_t off = uint32_t(kk) * 2u;  // 32 B in 16-byte units
+          mma_tf32_ss(tmem, ahi + off, bhi + off, idesc, (c | kk) != 0 ? 1u : 0u);
+          mma_tf32_ss(tmem, ahi + off, blo + off, idesc, 1u);
+          mma_tf32_ss(tmem, alo + off, bhi + off, idesc, 1u);
+        }
+        mma_commit(&sm.empty[s]);
+      }
+      if (ok) {
+        mma_commit(&sm.acc_full);
+      } else {
+        fail_status(a.status, &sm.abort, kDevErrTimeoutMma);
+        mma_commit(&sm.acc_full);  // lets the epilogue and the CTA end (bounded)
+        int never = 0;
+        mbar_wait(&sm.acc_full, 0, &never);
+      }
+    }
+  } else {
+    // epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 = tile rows
+    const int quad = warp & 3;
+    const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sm.acc_full, 0, abort)) && !*abort;
+    if (ok) {
+      tc_fence_after_sync();
+      float* stage = &sm.a[0][0][0] + size_t(warp - 2) * 32 * kLtStagePitch;
+      const uint32_t t_row = tmem + (uint32_t(quad * 32) << 16);
 #pragma unroll 1
-  for (int c = 0; c < kSlices; ++c) {
-    const int cur = c & 1;
-    if (c + 1 < kSlices) {
-      load_slice<D>(qa, g.nb, r0, (c + 1) * kBK, ra);
-      load_slice<D>(kb, g.nb, c0, (c + 1) * kBK, rb);
-    }
-    const float* A = As + cur * kBK * kLds + ty * 8;
-    const float* Bm = Bs + cur * kBK * kLds + tx * 4;
-#pragma unroll 8
-    for (int k = 0; k < kBK; ++k) {
-      const float4 a0 = *reinterpret_cast<const float4*>(A + k * kLds);
-      const float4 a1 = *reinterpret_cast<const float4*>(A + k * kLds + 4);
-      const float4 b0 = *reinterpret_cast<const float4*>(Bm + k * kLds);
-      const float4 b1 = *reinterpret_cast<const float4*>(Bm + k * kLds + 64);
-      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+      for (int cc = 0; cc < kLtN / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(t_row + 32 * cc, v);
+        tmem_wait_ld();
+        float4* dst = reinterpret_cast<float4*>(stage + lane * kLtStagePitch + 32 * cc);
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-    }
-    if (c + 1 < kSlices) {
-      store_slice(As + (cur ^ 1) * kBK * kLds, ra);
-      store_slice(Bs + (cur ^ 1) * kBK * kLds, rb);
-    }
-    __syncthreads();
-  }
-  float* out = L + size_t(bh) * g.nb * ld;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int r = r0 + ty * 8 + i;
-    if (r < g.nb) {
-      float* dst = out + size_t(r) * ld + c0 + tx * 4;
-      *reinterpret_cast<float4*>(dst) = make_float4(acc[i][0] * scale, acc[i][1] * scale,
-                                                    acc[i][2] * scale, acc[i][3] * scale);
-      *reinterpret_cast<float4*>(dst + 64) = make_float4(acc[i][4] * scale, acc[i][5] * scale,
-                                                         acc[i][6] * scale, acc[i][7] * scale);
+        for (int i = 0; i < 8; ++i)
+          dst[i] = make_float4(__uint_as_float(v[4 * i]) * a.scale,
+                               __uint_as_float(v[4 * i + 1]) * a.scale,
+                               __uint_as_float(v[4 * i + 2]) * a.scale,
+                               __uint_as_float(v[4 * i + 3]) * a.scale);
+      }
+      __syncwarp();
+      // row by row: the warp writes 1 KB contiguous per row
+      for (int rr = 0; rr < 32; ++rr) {
+        const int row = r0 + quad * 32 + rr;
+        if (row >= g.nb) break;  // rows ascend with rr
+        const float* src = stage + rr * kLtStagePitch;
+        float* out = a.logits + (size_t(row_base) + row) * ld + c0;
+        reinterpret_cast<float4*>(out)[lane] = reinterpret_cast<const float4*>(src)[lane];
+        reinterpret_cast<float4*>(out + 128)[lane] = reinterpret_cast<const float4*>(src + 128)[lane];
+      }
     }
   }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  if (warp == 1) tmem_dealloc(tmem, 256);
 }
 
 // ------------------------------------------------------------------ select
@@ -484,13 +533,12 @@ cudaError_t launch_select(const MaskArgs& a, const Geometry& g, int ld, cudaStre
 
 template <int D>
 cudaError_t launch_logits(const MaskArgs& a, const Geometry& g, int ld, cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(logits_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(kLogitSmem));
+  const int smem = int(sizeof(LogitsSmem) + 1024);
+  cudaError_t e = cudaFuncSetAttribute(logits_tc_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const dim3 grid(unsigned(ld / kBN), unsigned((g.nb + kBM - 1) / kBM), unsigned(g.BH));
-  logits_kernel<D><<<grid, kLogitThreads, kLogitSmem, stream>>>(a.qbar, a.kbar, a.logits, g, ld,
-                                                                a.scale);
+  const dim3 grid(unsigned(ld / kLtN), unsigned((g.nb + kLtM - 1) / kLtM), unsigned(g.BH));
+  logits_tc_kernel<D><<<grid, kLtThreads, smem, stream>>>(a, g, ld);
   return cudaGetLastError();
 }
 

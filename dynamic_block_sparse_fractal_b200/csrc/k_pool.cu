@@ -5,7 +5,11 @@
 //
 // One warp per (bh, block) and tensor; each lane owns d/32 channels and
 // streams the 64 token rows with coalesced 8-byte (d = 128) or 4-byte loads,
-// accumulating in fp32. HBM-bound: reads Q and K once, writes Qbar, Kbar.
+// accumulating in fp32. HBM-bound: reads Q and K once, writes Qbar, Kbar and
+// their split hi = tf32(x) (round to nearest, ties away), lo = x - hi (exact
+// in fp32), which the logits GEMM multiplies as hi*hi + hi*lo + lo*hi on the
+// TF32 tensor cores: the dropped lo*lo term and the tf32 rounding of lo are
+// both ~2^-22 relative, fp32-level accuracy.
 #include <cuda_bf16.h>
 
 #include "kernels.cuh"
@@ -16,7 +20,9 @@ template <int D>
 __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ q,
                                                    const __nv_bfloat16* __restrict__ k,
                                                    float* __restrict__ qbar,
-                                                   float* __restrict__ kbar, Geometry g) {
+                                                   float* __restrict__ kbar,
+                                                   float* __restrict__ qsplit,
+                                                   float* __restrict__ ksplit, Geometry g) {
   constexpr int kPerLane = D / 32;  // 4 or 2 channels per lane
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long unit = long(blockIdx.x) * 8 + warp;  // (tensor, bh, b)
@@ -56,22 +62,32 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
       }
     }
   }
-  float* dst = (which == 0 ? qbar : kbar) + (size_t(bh) * g.nb + b) * D + lane * kPerLane;
+  const size_t off = (size_t(bh) * g.nb + b) * D + lane * kPerLane;
+  const size_t half = size_t(g.BH) * g.nb * D;  // lo follows hi
+  float* dst = (which == 0 ? qbar : kbar) + off;
+  float* hi = (which == 0 ? qsplit : ksplit) + off;
   const float inv = 1.0f / 64.0f;  // exact: N = 64
 #pragma unroll
-  for (int i = 0; i < kPerLane; ++i) dst[i] = acc[i] * inv;
+  for (int i = 0; i < kPerLane; ++i) {
+    const float x = acc[i] * inv;
+    uint32_t h;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(x));
+    dst[i] = x;
+    hi[i] = __uint_as_float(h);
+    hi[half + i] = x - __uint_as_float(h);
+  }
 }
 
-cudaError_t launch_pool(const void* q, const void* k, float* qbar, float* kbar, const Geometry& g,
-                        cudaStream_t stream) {
+cudaError_t launch_pool(const void* q, const void* k, float* qbar, float* kbar, float* qsplit,
+                        float* ksplit, const Geometry& g, cudaStream_t stream) {
   const long units = 2L * g.BH * g.nb;
   const unsigned grid = unsigned((units + 7) / 8);
   const auto* qq = static_cast<const __nv_bfloat16*>(q);
   const auto* kk = static_cast<const __nv_bfloat16*>(k);
   if (g.d == 128)
-    pool_kernel<128><<<grid, 256, 0, stream>>>(qq, kk, qbar, kbar, g);
+    pool_kernel<128><<<grid, 256, 0, stream>>>(qq, kk, qbar, kbar, qsplit, ksplit, g);
   else
-    pool_kernel<64><<<grid, 256, 0, stream>>>(qq, kk, qbar, kbar, g);
+    pool_kernel<64><<<grid, 256, 0, stream>>>(qq, kk, qbar, kbar, qsplit, ksplit, g);
   return cudaGetLastError();
 }
 

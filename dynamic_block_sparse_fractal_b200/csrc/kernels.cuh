@@ -10,8 +10,10 @@
 
 namespace sa {
 
-cudaError_t launch_pool(const void* q, const void* k, float* qbar, float* kbar, const Geometry& g,
-                        cudaStream_t stream);
+// Qbar, Kbar (fp32 means) and their tf32 hi / lo split for the logits GEMM
+// (qsplit, ksplit: [2][BH][nb][d], hi first).
+cudaError_t launch_pool(const void* q, const void* k, float* qbar, float* kbar, float* qsplit,
+                        float* ksplit, const Geometry& g, cudaStream_t stream);
 
 cudaError_t launch_permute(const void* x, void* y, const Geometry& g, int inverse,
                            cudaStream_t stream);
@@ -20,6 +22,8 @@ cudaError_t launch_permute(const void* x, void* y, const Geometry& g, int invers
 // bitmaps, then per-tile union lists. target_fx = round((1 - thr) * 2^30)
 // (mass threshold in the select kernel's fixed point); dense = (thr == 0).
 struct MaskArgs {
+  CUtensorMap map_qhi, map_qlo;  // [BH*nb][d] fp32, box 32 x 128 rows
+  CUtensorMap map_khi, map_klo;  // [BH*nb][d] fp32, box 32 x 256 rows
   const float* qbar;
   const float* kbar;
   float* logits;   // [BH][nb][logits_ld(g)]
@@ -28,6 +32,7 @@ struct MaskArgs {
   int32_t* idx;
   int32_t* tcnt;
   int32_t* tidx;
+  uint32_t* status;  // device status word (bounded waits of the logits GEMM)
   uint32_t target_fx;
   int dense;
   int sta_t, sta_h, sta_w;  // half-widths (window / 2), -1 = no STA

@@ -74,14 +74,16 @@ struct WsLayout {
   size_t tcnt;     // int32 [BH][ntile]
   size_t tidx;     // int32 [BH][ntile][nb]
   size_t order;    // int32 [BH][ntile]: tiles of a head, heaviest union first
+  size_t qsplit;   // float [2][BH][nb][d]: Qbar as tf32 hi and lo = Qbar - hi
+  size_t ksplit;   // float [2][BH][nb][d]: the same for Kbar
   size_t logits;   // float [BH][nb][logits_ld]: the reduced map's scaled logits
   size_t bits;     // uint32 [BH][nb][nwords]: keep bitmap of every q-block row
   size_t total;
 };
 
-// Row pitch of the logits region (whole 128-column tiles of the logits GEMM)
+// Row pitch of the logits region (whole 256-column tiles of the logits GEMM)
 // and words per keep bitmap.
-SA_HD int logits_ld(const Geometry& g) { return (g.nb + 127) / 128 * 128; }
+SA_HD int logits_ld(const Geometry& g) { return (g.nb + 255) / 256 * 256; }
 SA_HD int bitmap_words(const Geometry& g) { return (g.nb + 31) / 32; }
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -97,6 +99,8 @@ inline WsLayout make_ws_layout(const Geometry& g) {
   w.tcnt = o; o = align256(o + sizeof(int32_t) * size_t(g.BH) * g.ntile);
   w.tidx = o; o = align256(o + sizeof(int32_t) * size_t(g.BH) * g.ntile * g.nb);
   w.order = o; o = align256(o + sizeof(int32_t) * size_t(g.BH) * g.ntile);
+  w.qsplit = o; o = align256(o + sizeof(float) * 2 * size_t(g.BH) * g.nb * g.d);
+  w.ksplit = o; o = align256(o + sizeof(float) * 2 * size_t(g.BH) * g.nb * g.d);
   w.logits = o; o = align256(o + sizeof(float) * size_t(g.BH) * g.nb * logits_ld(g));
   w.bits = o; o = align256(o + sizeof(uint32_t) * size_t(g.BH) * g.nb * bitmap_words(g));
   w.total = o;

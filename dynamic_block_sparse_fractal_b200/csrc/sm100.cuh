@@ -280,6 +280,27 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, in
 // sbo is the byte stride between 8-row groups; for MN-major operands lbo is
 // the stride between 64-element column chunks and sbo the stride between
 // groups of 8 K-rows.
+// Instruction descriptor, kind::tf32 with TF32 A/B (format code 2, as the
+// CUTLASS UMMA descriptor defines it) and fp32 D, both operands K-major.
+__host__ __device__ constexpr uint32_t idesc_tf32_f32(int M, int N) {
+  return (1u << 4)                            // D format: f32
+         | (2u << 7)                          // A format: tf32
+         | (2u << 10)                         // B format: tf32
+         | (uint32_t(N >> 3) << 17)           // N / 8
+         | (uint32_t(M >> 4) << 24);          // M / 16
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T on 32-bit TF32 operands (K = 8 per MMA).
+__device__ __forceinline__ void mma_tf32_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   return uint64_t((saddr & 0x3FFFFu) >> 4) | (uint64_t((lbo >> 4) & 0x3FFFu) << 16) |
          (uint64_t((sbo >> 4) & 0x3FFFu) << 32) | (uint64_t(1) << 46)  // sm100 descriptor

@@ -44,4 +44,22 @@ inline bool encode_patch_map(CUtensorMap* map, const void* base, int BH, int T, 
   return r == CUDA_SUCCESS;
 }
 
+// fp32 matrix [rows][cols] (cols innermost, cols * 4 a multiple of 16 bytes)
+// seen as a 2-D TMA tensor whose box is 32 columns (128 bytes) x box_rows
+// rows, written to shared memory with the 128-byte swizzle; rows or columns
+// past the end read as zeros. Coordinates are (column, row).
+inline bool encode_rows_f32(CUtensorMap* map, const void* base, long long rows, int cols,
+                            int box_rows) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(cols) * 4};
+  cuuint32_t box[2] = {32, cuuint32_t(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace sa
