@@ -16,6 +16,14 @@ notes as well):
 
 * Fractal order: time outermost, then patch row, then patch column; inside a
   P x P patch the tokens are row-major (h % P, then w % P).
+* Three-dimensional tiles (the head-aware tiling of "Veda" on the page
+  "Veda: Video Generation with Efficient Sparse Attention", section 2.2,
+  "Tiling Consapevole delle Teste"): a tile shape (p_t, p_h, p_w) with
+  p_t * p_h * p_w = N makes each block p_t consecutive frames of a
+  p_h x p_w patch. Blocks are ordered (t // p_t, h // p_h, w // p_w) and the
+  tokens inside a block (t % p_t, h % p_h, w % p_w), both row-major; the
+  square patch of one frame is the shape (1, P, P). Block coordinates and the
+  STA window are then in units of blocks along each axis.
 * Pooling "in N x N blocks" means the mean of N consecutive tokens of the
   reordered sequence; the N x N refers to the block of the attention map.
 * The reduced map uses the same 1/sqrt(d) scale as the main attention and no
@@ -40,22 +48,35 @@ def widen_bf16(bits: np.ndarray) -> np.ndarray:
 
 # --- Metodologia 1: "Riordinamento dei Token (Fractal Flattening)" ----------
 
-def fractal_order(T: int, Hh: int, Ww: int, P: int) -> np.ndarray:
+def tile_shape(P) -> tuple:
+    """(p_t, p_h, p_w) of a block: an int P is the P x P patch of one frame."""
+    if isinstance(P, (tuple, list)):
+        pt, ph, pw = (int(v) for v in P)
+        return pt, ph, pw
+    return 1, int(P), int(P)
+
+
+def fractal_order(T: int, Hh: int, Ww: int, P) -> np.ndarray:
     """perm[i] = natural-order index of the token at position i of the
     fractally flattened sequence.
 
-    Tokens of each P x P spatial patch become contiguous; frames stay in
-    time order. Natural order index of (t, h, w) is t*Hh*Ww + h*Ww + w.
-    Position order is (t, patch row hp, patch column wp, h % P, w % P).
+    Tokens of each block (a P x P spatial patch of one frame, or a
+    p_t x p_h x p_w tile) become contiguous; blocks and the frames inside a
+    block stay in time order. Natural order index of (t, h, w) is
+    t*Hh*Ww + h*Ww + w. Position order is (t // p_t, h // p_h, w // p_w,
+    t % p_t, h % p_h, w % p_w).
     """
-    if Hh % P or Ww % P:
-        raise ValueError("Hh and Ww must be multiples of P")
-    t = np.arange(T).reshape(T, 1, 1, 1, 1)
-    hp = np.arange(Hh // P).reshape(1, Hh // P, 1, 1, 1)
-    wp = np.arange(Ww // P).reshape(1, 1, Ww // P, 1, 1)
-    hi = np.arange(P).reshape(1, 1, 1, P, 1)
-    wi = np.arange(P).reshape(1, 1, 1, 1, P)
-    natural = t * (Hh * Ww) + (hp * P + hi) * Ww + (wp * P + wi)
+    pt, ph, pw = tile_shape(P)
+    if T % pt or Hh % ph or Ww % pw:
+        raise ValueError("T, Hh, Ww must be multiples of the tile shape")
+    nt, nh, nw = T // pt, Hh // ph, Ww // pw
+    tb = np.arange(nt).reshape(nt, 1, 1, 1, 1, 1)
+    hb = np.arange(nh).reshape(1, nh, 1, 1, 1, 1)
+    wb = np.arange(nw).reshape(1, 1, nw, 1, 1, 1)
+    ti = np.arange(pt).reshape(1, 1, 1, pt, 1, 1)
+    hi = np.arange(ph).reshape(1, 1, 1, 1, ph, 1)
+    wi = np.arange(pw).reshape(1, 1, 1, 1, 1, pw)
+    natural = (tb * pt + ti) * (Hh * Ww) + (hb * ph + hi) * Ww + (wb * pw + wi)
     return natural.reshape(-1).astype(np.int64)
 
 
@@ -115,16 +136,18 @@ def cdf_keep(A: np.ndarray, thr: float) -> np.ndarray:
     return keep
 
 
-def block_coords(T: int, Hh: int, Ww: int, P: int) -> np.ndarray:
-    """(t, hp, wp) of every block in fractal order when N = P*P, shape [nb, 3]."""
-    nh, nw = Hh // P, Ww // P
-    b = np.arange(T * nh * nw)
+def block_coords(T: int, Hh: int, Ww: int, P) -> np.ndarray:
+    """(t, hp, wp) of every block in fractal order, in block units
+    (t // p_t, h // p_h, w // p_w), shape [nb, 3]."""
+    pt, ph, pw = tile_shape(P)
+    nt, nh, nw = T // pt, Hh // ph, Ww // pw
+    b = np.arange(nt * nh * nw)
     return np.stack([b // (nh * nw), (b // nw) % nh, b % nw], axis=1)
 
 
 # --- Metodologia 3: "Integrazione Ibrida con STA" ---------------------------
 
-def sta_keep(T: int, Hh: int, Ww: int, P: int, sta) -> np.ndarray:
+def sta_keep(T: int, Hh: int, Ww: int, P, sta) -> np.ndarray:
     """Static sliding-tile window in block units: q-block and k-block are
     paired iff their distance along each of (t, hp, wp) is at most half the
     (odd) window size. (0, 0, 0) is no window. [nb, nb] bool."""
@@ -156,8 +179,9 @@ def nabla_mask(q, k, T, Hh, Ww, P, N, thr, sta):
     one head at a time. Returns (M, M_nabla, A): bool [BH, nb, nb] masks and
     the float64 reduced map.
     """
-    if N != P * P:
-        raise ValueError("this reading needs N == P*P (one block = one patch)")
+    pt, ph, pw = tile_shape(P)
+    if N != pt * ph * pw:
+        raise ValueError("this reading needs N == p_t * p_h * p_w (one block = one tile)")
     m_sta = sta_keep(T, Hh, Ww, P, sta)
     BH, nb = q.shape[0], q.shape[1] // N
     A = np.empty((BH, nb, nb))

@@ -138,6 +138,16 @@ def pin_attention_own_patch():
 
 # --- the pins as tests -------------------------------------------------------
 
+def pin_fractal_reshape_3d(T=4, Hh=8, Ww=16, tile=(2, 4, 8)):
+    # Independent construction for a p_t x p_h x p_w tile: view the natural
+    # index grid as [T/pt, pt, Hh/ph, ph, Ww/pw, pw] and move the three
+    # in-tile axes innermost, in (t, h, w) order.
+    pt, ph, pw = tile
+    idx = np.arange(T * Hh * Ww).reshape(T // pt, pt, Hh // ph, ph, Ww // pw, pw)
+    expect = idx.transpose(0, 2, 4, 1, 3, 5).reshape(-1)
+    assert np.array_equal(oracle.fractal_order(T, Hh, Ww, tile), expect)
+
+
 def test_fractal_order_golden(golden_dir):
     pin_fractal_golden(golden_dir)
 
@@ -161,6 +171,72 @@ def test_fractal_round_trip_and_patches():
         assert len(set(t[sl])) == 1 and len(set(h[sl] // P)) == 1 and len(set(w[sl] // P)) == 1
         assert len(set(zip(h[sl], w[sl]))) == P * P
     assert np.array_equal(t, np.sort(t))  # time stays ordered
+
+
+def test_fractal_order_3d_tiles_match_reshape():
+    pin_fractal_reshape_3d()
+    pin_fractal_reshape_3d(T=8, Hh=16, Ww=16, tile=(4, 4, 4))
+    pin_fractal_reshape_3d(T=3, Hh=8, Ww=32, tile=(1, 4, 16))
+    # the square patch of one frame is the tile (1, P, P)
+    assert np.array_equal(oracle.fractal_order(3, 16, 24, (1, 8, 8)),
+                          oracle.fractal_order(3, 16, 24, 8))
+
+
+def test_fractal_3d_round_trip_and_tiles():
+    T, Hh, Ww, tile = 8, 8, 16, (2, 4, 8)
+    pt, ph, pw = tile
+    n = pt * ph * pw
+    perm = oracle.fractal_order(T, Hh, Ww, tile)
+    assert np.array_equal(np.sort(perm), np.arange(T * Hh * Ww))
+    t, h, w = perm // (Hh * Ww), (perm // Ww) % Hh, perm % Ww
+    coords = oracle.block_coords(T, Hh, Ww, tile)
+    for b in range(perm.size // n):
+        sl = slice(b * n, (b + 1) * n)
+        # each run of N positions is exactly one p_t x p_h x p_w tile ...
+        assert set(zip(t[sl], h[sl], w[sl])) == {
+            (coords[b, 0] * pt + i, coords[b, 1] * ph + j, coords[b, 2] * pw + k)
+            for i in range(pt) for j in range(ph) for k in range(pw)}
+    # ... and block coordinates ascend in (t, h, w) block order
+    nt, nh, nw = T // pt, Hh // ph, Ww // pw
+    assert [tuple(c) for c in coords] == [(a, b, c) for a in range(nt) for b in range(nh)
+                                          for c in range(nw)]
+
+
+def test_sta_3d_tiles_loop():
+    T, Hh, Ww, tile, win = 8, 8, 16, (2, 4, 4), (3, 1, 3)
+    pt, ph, pw = tile
+    nt, nh, nw = T // pt, Hh // ph, Ww // pw
+    got = oracle.sta_keep(T, Hh, Ww, tile, win)
+    expect = np.zeros((nt * nh * nw,) * 2, dtype=bool)
+    for t1, h1, w1 in itertools.product(range(nt), range(nh), range(nw)):
+        for t2, h2, w2 in itertools.product(range(nt), range(nh), range(nw)):
+            if abs(t1 - t2) <= 1 and h1 == h2 and abs(w1 - w2) <= 1:
+                expect[(t1 * nh + h1) * nw + w1, (t2 * nh + h2) * nw + w2] = True
+    assert np.array_equal(got, expect)
+
+
+def pin_attention_own_tile_3d():
+    # One kept block per row (the query's own tile): each output is plain
+    # attention over the tokens of the query's p_t x p_h x p_w tile, computed
+    # here from token coordinates alone.
+    rng = np.random.default_rng(23)
+    T, Hh, Ww, tile = 4, 8, 8, (2, 4, 8)
+    pt, ph, pw = tile
+    S, d = T * Hh * Ww, 8
+    q, k, v = (rng.standard_normal((S, d)) for _ in range(3))
+    nb = S // (pt * ph * pw)
+    out = oracle.attention_head(q, k, v, T, Hh, Ww, tile, pt * ph * pw, np.eye(nb, dtype=bool))
+    t, h, w = np.arange(S) // (Hh * Ww), (np.arange(S) // Ww) % Hh, np.arange(S) % Ww
+    key = (t // pt) * 1000000 + (h // ph) * 1000 + (w // pw)
+    for i in (0, 5, 77, 200, 255):
+        cols = np.nonzero(key == key[i])[0]
+        s_ = q[i] @ k[cols].T / np.sqrt(d)
+        e = np.exp(s_ - s_.max())
+        assert np.abs(out[i] - e @ v[cols] / e.sum()).max() < 1e-12
+
+
+def test_attention_3d_tile_single_block_is_tile_attention():
+    pin_attention_own_tile_3d()
 
 
 def test_pool_closed_forms():
@@ -292,6 +368,18 @@ def _mut_fractal_patch_col_major(T, Hh, Ww, P):
     return idx.transpose(0, 3, 1, 2, 4).reshape(-1)
 
 
+def _mut_fractal3d_tile_w_before_h(T, Hh, Ww, P):
+    pt, ph, pw = nabla.tile_shape(P)
+    idx = np.arange(T * Hh * Ww).reshape(T // pt, pt, Hh // ph, ph, Ww // pw, pw)
+    return idx.transpose(0, 2, 4, 1, 5, 3).reshape(-1)
+
+
+def _mut_fractal3d_time_inside_patch_last(T, Hh, Ww, P):
+    pt, ph, pw = nabla.tile_shape(P)
+    idx = np.arange(T * Hh * Ww).reshape(T // pt, pt, Hh // ph, ph, Ww // pw, pw)
+    return idx.transpose(0, 2, 4, 3, 5, 1).reshape(-1)
+
+
 def _mut_cdf_le(A, thr):
     if thr == 0.0:
         return np.ones(A.shape, dtype=bool)
@@ -361,6 +449,8 @@ _orig_masked = nabla.masked_attention
 MUTANTS = [
     ("fractal_order", _mut_fractal_inner_transposed, "fractal"),
     ("fractal_order", _mut_fractal_patch_col_major, "fractal"),
+    ("fractal_order", _mut_fractal3d_tile_w_before_h, "fractal3d"),
+    ("fractal_order", _mut_fractal3d_time_inside_patch_last, "fractal3d"),
     ("cdf_keep", _mut_cdf_le, "cdf"),
     ("cdf_keep", _mut_cdf_ascending, "cdf"),
     ("cdf_keep", _mut_cdf_threshold_is_thr, "cdf"),
@@ -379,6 +469,7 @@ def test_planted_mistake_is_caught(name, mutant, area, golden_dir, monkeypatch):
     monkeypatch.setattr(oracle, name, mutant)
     pins = {
         "fractal": [lambda: pin_fractal_golden(golden_dir), pin_fractal_reshape],
+        "fractal3d": [pin_fractal_reshape_3d, pin_attention_own_tile_3d],
         "cdf": [lambda: pin_cdf_golden(golden_dir), pin_cdf_bruteforce],
         "reduced": [pin_reduced_closed_form],
         "sta": [lambda: pin_sta_golden(golden_dir)],
