@@ -333,11 +333,11 @@ def oracle_sample(w, budget_s=20.0, seed=0):
     heads = [0]
     q, k, v = W.make_inputs(w, heads=range(0, 1))
     t = time.perf_counter()
-    M, _, _ = oracle.nabla_mask(q, k, w.T, w.Hh, w.Ww, w.P, w.N, w.thr, w.sta)
+    M, _, _ = oracle.nabla_mask(q, k, w.T, w.Hh, w.Ww, w.block, w.N, w.thr, w.sta)
     mask_s = time.perf_counter() - t
     rng = np.random.default_rng(seed)
     order = rng.permutation(w.nb)
-    perm = oracle.fractal_order(w.T, w.Hh, w.Ww, w.P)
+    perm = oracle.fractal_order(w.T, w.Hh, w.Ww, w.block)
     qp, kp, vp = (oracle.flatten(oracle.widen_bf16(x[0]), perm) for x in (q, k, v))
     pairs, spent, nq = 0, 0.0, 0
     t = time.perf_counter()

@@ -36,7 +36,8 @@ class SaDesc(ctypes.Structure):
                 ("Hh", ctypes.c_int), ("Ww", ctypes.c_int), ("d", ctypes.c_int),
                 ("N", ctypes.c_int), ("P", ctypes.c_int), ("thr", ctypes.c_float),
                 ("sta_t", ctypes.c_int), ("sta_h", ctypes.c_int), ("sta_w", ctypes.c_int),
-                ("out_fp32", ctypes.c_int), ("debug_flags", ctypes.c_int)]
+                ("out_fp32", ctypes.c_int), ("debug_flags", ctypes.c_int),
+                ("pt", ctypes.c_int), ("ph", ctypes.c_int), ("pw", ctypes.c_int)]
 
 
 class SaMaskViews(ctypes.Structure):
@@ -93,15 +94,18 @@ def _ok(status: int, what: str) -> None:
 
 def make_desc(B: int, H: int, T: int, Hh: int, Ww: int, d: int, thr: float,
               sta=(0, 0, 0), N: int = 64, P: int = 8, out_fp32: bool = False,
-              debug_flags: int = 0) -> SaDesc:
+              debug_flags: int = 0, tile=None) -> SaDesc:
+    """tile: block shape (pt, ph, pw) with pt*ph*pw == N, or None for the
+    P x P patch of one frame."""
+    pt, ph, pw = (0, 0, 0) if tile is None else (int(v) for v in tile)
     return SaDesc(B, H, T, Hh, Ww, d, N, P, float(thr), int(sta[0]), int(sta[1]), int(sta[2]),
-                  int(bool(out_fp32)), int(debug_flags))
+                  int(bool(out_fp32)), int(debug_flags), pt, ph, pw)
 
 
 def desc_for(w, out_fp32: bool = False, debug_flags: int = 0) -> SaDesc:
     """Descriptor of a workload from ``workloads``."""
     return make_desc(w.B, w.H, w.T, w.Hh, w.Ww, w.d, w.thr, w.sta, w.N, w.P, out_fp32,
-                     debug_flags)
+                     debug_flags, getattr(w, "tile", None))
 
 
 def _stream(stream) -> ctypes.c_void_p:
@@ -211,8 +215,9 @@ class NablaAttention:
     """User-facing wrapper: owns a workspace; ``plan`` builds the block mask,
     ``forward`` runs the block-sparse attention; calling it does both."""
 
-    def __init__(self, B, H, T, Hh, Ww, d, thr, sta=(0, 0, 0), out_fp32=False, device="cuda"):
-        self.desc = make_desc(B, H, T, Hh, Ww, d, thr, sta, out_fp32=out_fp32)
+    def __init__(self, B, H, T, Hh, Ww, d, thr, sta=(0, 0, 0), out_fp32=False, device="cuda",
+                 tile=None):
+        self.desc = make_desc(B, H, T, Hh, Ww, d, thr, sta, out_fp32=out_fp32, tile=tile)
         self.workspace = alloc_workspace(self.desc, device)
 
     def plan(self, q, k, stream=None):

@@ -23,8 +23,9 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 sa_status validate(const sa_desc* d) {
   if (d == nullptr) return SA_ERR_INVALID_ARG;
+  const bool tiled = d->pt != 0 || d->ph != 0 || d->pw != 0;
   if (d->B < 1 || d->H < 1 || d->T < 1 || d->Hh < 1 || d->Ww < 1 || d->d < 1 || d->N < 1 ||
-      d->P < 1)
+      (!tiled && d->P < 1))
     return SA_ERR_INVALID_ARG;
   if (!(d->thr >= 0.0f && d->thr < 1.0f)) return SA_ERR_INVALID_ARG;  // also rejects NaN
   const bool no_sta = d->sta_t == 0 && d->sta_h == 0 && d->sta_w == 0;
@@ -35,10 +36,18 @@ sa_status validate(const sa_desc* d) {
   if (d->out_fp32 != 0 && d->out_fp32 != 1) return SA_ERR_INVALID_ARG;
   if (d->debug_flags & ~SA_DEBUG_STALL_LOADER) return SA_ERR_INVALID_ARG;
   if (d->d != 64 && d->d != 128) return SA_ERR_UNSUPPORTED;
-  if (d->P != 8 || d->N != d->P * d->P) return SA_ERR_UNSUPPORTED;
-  if (d->Hh % d->P || d->Ww % d->P) return SA_ERR_UNSUPPORTED;
+  if (d->N != 64) return SA_ERR_UNSUPPORTED;  // the attention kernel's 64-row blocks
+  int pt = 1, ph = d->P, pw = d->P;
+  if (tiled) {
+    if (d->pt < 1 || d->ph < 1 || d->pw < 1) return SA_ERR_INVALID_ARG;
+    pt = d->pt;
+    ph = d->ph;
+    pw = d->pw;
+  }
+  if ((long long)pt * ph * pw != d->N) return SA_ERR_UNSUPPORTED;  // also: powers of 2
+  if (d->T % pt || d->Hh % ph || d->Ww % pw) return SA_ERR_UNSUPPORTED;
   const long long BH = (long long)d->B * d->H;
-  const long long nb = (long long)d->T * (d->Hh / d->P) * (d->Ww / d->P);
+  const long long nb = (long long)(d->T / pt) * (d->Hh / ph) * (d->Ww / pw);
   if (BH > 65535 || nb > kMaxBlocks) return SA_ERR_UNSUPPORTED;
   return SA_OK;
 }
@@ -135,11 +144,12 @@ sa_status sparse_attn_fwd(const sa_desc* desc, const void* q, const void* k, con
   const WsLayout w = make_ws_layout(g);
   AttnArgs a;
   std::memset(&a, 0, sizeof(a));
-  if (!encode_patch_map(&a.map_q, q, g.BH, g.T, g.Hh, g.Ww, g.d, g.P) ||
-      !encode_patch_map(&a.map_k, k, g.BH, g.T, g.Hh, g.Ww, g.d, g.P) ||
-      !encode_patch_map(&a.map_v, v, g.BH, g.T, g.Hh, g.Ww, g.d, g.P) ||
-      !encode_patch_map(&a.map_k2, k, g.BH, g.T, g.Hh, g.Ww, g.d, g.P, g.T > 1 ? 2 : 1) ||
-      !encode_patch_map(&a.map_v2, v, g.BH, g.T, g.Hh, g.Ww, g.d, g.P, g.T > 1 ? 2 : 1))
+  const int pair_frames = g.nt > 1 ? 2 : 1;  // a temporal pair = two block frames
+  if (!encode_tile_map(&a.map_q, q, g.BH, g.T, g.Hh, g.Ww, g.d, g.pt, g.ph, g.pw) ||
+      !encode_tile_map(&a.map_k, k, g.BH, g.T, g.Hh, g.Ww, g.d, g.pt, g.ph, g.pw) ||
+      !encode_tile_map(&a.map_v, v, g.BH, g.T, g.Hh, g.Ww, g.d, g.pt, g.ph, g.pw) ||
+      !encode_tile_map(&a.map_k2, k, g.BH, g.T, g.Hh, g.Ww, g.d, g.pt, g.ph, g.pw, pair_frames) ||
+      !encode_tile_map(&a.map_v2, v, g.BH, g.T, g.Hh, g.Ww, g.d, g.pt, g.ph, g.pw, pair_frames))
     return SA_ERR_CUDA;
   a.out = out;
   a.tcnt = at<int32_t>(workspace, w.tcnt);

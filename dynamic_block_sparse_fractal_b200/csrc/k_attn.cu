@@ -226,8 +226,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             int t, hp, wp;
             block_coords(g, blk, t, hp, wp);
             for (int c = 0; c < D / 64; ++c)
-              tma_load_5d(&sm.q[x][c][e * 8192], &a.map_q, &sm.q_full[x], c * 64, wp * 8, hp * 8,
-                          t, bh);
+              tma_load_5d(&sm.q[x][c][e * 8192], &a.map_q, &sm.q_full[x], c * 64, wp * g.pw, hp * g.ph,
+                          t * g.pt, bh);
           }
         }
       }
@@ -258,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           block_coords(g, e0 & kEntryBlockMask, tt, hp, wp);
           const CUtensorMap* map = kind == 0 ? &a.map_k2 : &a.map_v2;
           for (int c = 0; c < D / 64; ++c)
-            tma_load_5d(&sm.slot[s][c][0], map, &sm.full[s], c * 64, wp * 8, hp * 8, tt, bh);
+            tma_load_5d(&sm.slot[s][c][0], map, &sm.full[s], c * 64, wp * g.pw, hp * g.ph, tt * g.pt, bh);
         } else {
           const CUtensorMap* map = kind == 0 ? &a.map_k : &a.map_v;
           for (int e = 0; e < nblk; ++e) {
@@ -270,8 +270,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             int tt, hp, wp;
             block_coords(g, kb, tt, hp, wp);
             for (int c = 0; c < D / 64; ++c)
-              tma_load_5d(&sm.slot[s][c][e * 8192], map, &sm.full[s], c * 64, wp * 8, hp * 8, tt,
-                          bh);
+              tma_load_5d(&sm.slot[s][c][e * 8192], map, &sm.full[s], c * 64, wp * g.pw, hp * g.ph,
+                          tt * g.pt, bh);
           }
         }
         last_issued = k;
@@ -509,9 +509,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int blk = half ? t.qb : t.qa;
           int tt, hp, wp;
           block_coords(g, blk, tt, hp, wp);
+          // row i of the block: frame tt*pt + (i >> (lph + lpw)), row
+          // hp*ph + ((i >> lpw) & (ph - 1)), column wp*pw + (i & (pw - 1))
           const int i = r & 63;
-          const size_t tok = size_t(tt) * g.Hh * g.Ww + size_t(hp * 8 + (i >> 3)) * g.Ww +
-                             size_t(wp * 8 + (i & 7));
+          const int run = i >> g.lpw;
+          const size_t tok = (size_t(tt) * g.pt + (run >> g.lph)) * g.Hh * g.Ww +
+                             size_t(hp * g.ph + (run & (g.ph - 1))) * g.Ww +
+                             size_t(wp * g.pw + (i & (g.pw - 1)));
           const size_t row = size_t(bh) * g.S + tok;
           const float inv = l > 0.f ? 1.0f / l : 0.f;
 #pragma unroll

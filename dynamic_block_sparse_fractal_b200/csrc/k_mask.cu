@@ -382,7 +382,7 @@ __global__ void __launch_bounds__(kSelWarps * 32, VPL <= 32 ? 4 : (VPL <= 64 ? 2
   if (a.sta_t >= 0) {
     int tq, hq, wq;
     block_coords(g, qb, tq, hq, wq);
-    const int t0 = max(tq - a.sta_t, 0), t1 = min(tq + a.sta_t, g.T - 1);
+    const int t0 = max(tq - a.sta_t, 0), t1 = min(tq + a.sta_t, g.nt - 1);
     const int h0 = max(hq - a.sta_h, 0), h1 = min(hq + a.sta_h, g.nh - 1);
     const int w0 = max(wq - a.sta_w, 0), w1 = min(wq + a.sta_w, g.nw - 1);
     const int nw_ = w1 - w0 + 1, nhw = (h1 - h0 + 1) * nw_;
@@ -429,14 +429,14 @@ constexpr int kUnionMaxWarps = 8;
 // frame), the first blocks of the temporal pairs and the unpaired blocks.
 SA_HD int union_words_per_warp(const Geometry& g) {
   const int fw = (g.nh * g.nw + 31) / 32;
-  return 2 * (bitmap_words(g) + 1) + 2 * g.T * fw;
+  return 2 * (bitmap_words(g) + 1) + 2 * g.nt * fw;
 }
 
 __global__ void __launch_bounds__(kUnionMaxWarps * 32) union_kernel(MaskArgs a, Geometry g) {
   extern __shared__ uint32_t ush[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nwords = bitmap_words(g);
-  const int pf = g.nh * g.nw, fw = (pf + 31) >> 5, nf = g.T * fw;
+  const int pf = g.nh * g.nw, fw = (pf + 31) >> 5, nf = g.nt * fw;
   const long item = long(blockIdx.x) * (blockDim.x >> 5) + warp;  // (bh, tile)
   if (item >= long(g.BH) * g.ntile) return;
   const int bh = int(item / g.ntile), tile = int(item - long(bh) * g.ntile);
@@ -468,7 +468,7 @@ __global__ void __launch_bounds__(kUnionMaxWarps * 32) union_kernel(MaskArgs a, 
   // second of a pair becomes the second of a pair.
   for (int w = lane; w < fw; w += 32) {
     uint32_t prev_in = 0u, prev_pair = 0u;
-    for (int t = 0; t < g.T; ++t) {
+    for (int t = 0; t < g.nt; ++t) {
       const uint32_t in = frame_word(t, w);
       const uint32_t pair = prev_in & ~prev_pair & in;
       if (t > 0) {
@@ -478,8 +478,8 @@ __global__ void __launch_bounds__(kUnionMaxWarps * 32) union_kernel(MaskArgs a, 
       prev_in = in;
       prev_pair = pair;
     }
-    firstF[(g.T - 1) * fw + w] = 0u;
-    leftF[(g.T - 1) * fw + w] = prev_in & ~prev_pair;
+    firstF[(g.nt - 1) * fw + w] = 0u;
+    leftF[(g.nt - 1) * fw + w] = prev_in & ~prev_pair;
   }
   __syncwarp();
 

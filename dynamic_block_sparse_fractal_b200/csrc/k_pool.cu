@@ -1,7 +1,8 @@
 // Block pooling of Q and K ("Sottocampionamento", NABLA Metodologia 2):
-// Qbar[bh][b] = mean of the N = P*P tokens of block b, i.e. of the P x P
-// patch (hp, wp) of frame t, read straight from the natural layout (the
-// fractal flattening is only an addressing here).
+// Qbar[bh][b] = mean of the N = 64 tokens of block b, i.e. of the P x P
+// patch (hp, wp) of frame t, or of the pt x ph x pw tile (t, hp, wp) in block
+// units, read straight from the natural layout (the fractal flattening is
+// only an addressing here). A block is pt * ph runs of pw consecutive tokens.
 //
 // One warp per (bh, block) and tensor; each lane owns d/32 channels and
 // streams the 64 token rows with coalesced 8-byte (d = 128) or 4-byte loads,
@@ -37,23 +38,28 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
   float acc[kPerLane];
 #pragma unroll
   for (int i = 0; i < kPerLane; ++i) acc[i] = 0.f;
-  const size_t frame0 = size_t(t) * g.Hh * g.Ww;
-#pragma unroll 4
-  for (int hi = 0; hi < 8; ++hi) {
-    const size_t row0 = frame0 + size_t(hp * 8 + hi) * g.Ww + wp * 8;
+  // token r of the block: frame t*pt + (r >> (lph + lpw)), row hp*ph +
+  // ((r >> lpw) & (ph - 1)), column wp*pw + (r & (pw - 1))
+  const size_t base_tok = (size_t(t) * g.pt * g.Hh + size_t(hp) * g.ph) * g.Ww + size_t(wp) * g.pw;
+#pragma unroll 2
+  for (int r0 = 0; r0 < 64; r0 += 8) {
     float2 raw[8];
 #pragma unroll
-    for (int wi = 0; wi < 8; ++wi) {
-      const __nv_bfloat16* p = src + (row0 + wi) * D;
+    for (int u = 0; u < 8; ++u) {
+      const int r = r0 + u;
+      const int run = r >> g.lpw, wi = r & (g.pw - 1);
+      const int ti = run >> g.lph, hi = run & (g.ph - 1);
+      const __nv_bfloat16* p =
+          src + (base_tok + (size_t(ti) * g.Hh + hi) * g.Ww + wi) * D;
       if constexpr (kPerLane == 4) {
-        raw[wi] = __ldg(reinterpret_cast<const float2*>(p));
+        raw[u] = __ldg(reinterpret_cast<const float2*>(p));
       } else {
-        raw[wi].x = __ldg(reinterpret_cast<const float*>(p));
+        raw[u].x = __ldg(reinterpret_cast<const float*>(p));
       }
     }
 #pragma unroll
-    for (int wi = 0; wi < 8; ++wi) {
-      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[wi]);
+    for (int u = 0; u < 8; ++u) {
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
 #pragma unroll
       for (int i = 0; i < kPerLane / 2; ++i) {
         const float2 f = __bfloat1622float2(h[i]);
@@ -91,33 +97,37 @@ cudaError_t launch_pool(const void* q, const void* k, float* qbar, float* kbar, 
   return cudaGetLastError();
 }
 
-// Fractal flattening as an explicit copy: position p = b*64 + hi*8 + wi of a
-// head holds the natural token (t, hp*8 + hi, wp*8 + wi) of block b. One warp
-// per (bh, block, patch row hi): 8 tokens x d channels, 16-byte vectors.
+// Fractal flattening as an explicit copy: position b*64 + r of a head holds
+// token r of block b (see the pooling above for r -> (t, h, w)). One warp per
+// (bh, block, run of pw consecutive tokens): pw tokens x d channels,
+// 16-byte vectors.
 __global__ void __launch_bounds__(256) permute_kernel(const uint4* __restrict__ x,
                                                       uint4* __restrict__ y, Geometry g,
                                                       int inverse) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long unit = long(blockIdx.x) * 8 + warp;  // (bh, b, hi)
-  if (unit >= long(g.BH) * g.nb * 8) return;
-  const int hi = int(unit & 7);
-  const long bb = unit >> 3;
+  const int runs = 64 >> g.lpw;                   // pt * ph runs per block
+  const long unit = long(blockIdx.x) * 8 + warp;  // (bh, b, run)
+  if (unit >= long(g.BH) * g.nb * runs) return;
+  const long bb = unit / runs;
+  const int run = int(unit - bb * runs);
   const int bh = int(bb / g.nb), b = int(bb - long(bh) * g.nb);
   int t, hp, wp;
   block_coords(g, b, t, hp, wp);
+  const int ti = run >> g.lph, hi = run & (g.ph - 1);
   const int vec_per_row = g.d / 8;  // 16-byte vectors per token row
-  const size_t nat = size_t(t) * g.Hh * g.Ww + size_t(hp * 8 + hi) * g.Ww + wp * 8;
-  const size_t frac = size_t(b) * 64 + hi * 8;
+  const size_t nat = (size_t(t) * g.pt + ti) * g.Hh * g.Ww + size_t(hp * g.ph + hi) * g.Ww +
+                     size_t(wp) * g.pw;
+  const size_t frac = size_t(b) * 64 + size_t(run) * g.pw;
   const size_t head = size_t(bh) * g.S;
   const size_t src0 = (head + (inverse ? frac : nat)) * vec_per_row;
   const size_t dst0 = (head + (inverse ? nat : frac)) * vec_per_row;
-  // the 8 tokens of a patch row are contiguous in both orders
-  for (int i = lane; i < 8 * vec_per_row; i += 32) y[dst0 + i] = __ldg(x + src0 + i);
+  // the pw tokens of a run are contiguous in both orders
+  for (int i = lane; i < g.pw * vec_per_row; i += 32) y[dst0 + i] = __ldg(x + src0 + i);
 }
 
 cudaError_t launch_permute(const void* x, void* y, const Geometry& g, int inverse,
                            cudaStream_t stream) {
-  const long units = long(g.BH) * g.nb * 8;
+  const long units = long(g.BH) * g.nb * (64 >> g.lpw);
   permute_kernel<<<unsigned((units + 7) / 8), 256, 0, stream>>>(
       static_cast<const uint4*>(x), static_cast<uint4*>(y), g, inverse);
   return cudaGetLastError();

@@ -12,8 +12,10 @@ namespace sa {
 
 struct Geometry {
   int BH, T, Hh, Ww, d, P, N;
-  int nh, nw;   // patches per frame along h and w
-  int nb;       // blocks per head = T * nh * nw
+  int pt, ph, pw;     // block shape (frames, rows, columns); pt*ph*pw = N
+  int lph, lpw;       // log2(ph), log2(pw) (N = 64: every extent is a power of 2)
+  int nt, nh, nw;     // blocks along t, h and w
+  int nb;             // blocks per head = nt * nh * nw
   int ntile;    // query tiles per head
   int S;        // tokens per head
 };
@@ -26,17 +28,27 @@ SA_HD Geometry make_geometry(const sa_desc& s) {
   g.Ww = s.Ww;
   g.d = s.d;
   g.P = s.P;
+  const bool tiled = s.pt != 0 || s.ph != 0 || s.pw != 0;
+  g.pt = tiled ? s.pt : 1;
+  g.ph = tiled ? s.ph : s.P;
+  g.pw = tiled ? s.pw : s.P;
+  g.lph = 0;
+  while ((1 << g.lph) < g.ph) ++g.lph;
+  g.lpw = 0;
+  while ((1 << g.lpw) < g.pw) ++g.lpw;
   g.N = s.N;
-  g.nh = s.Hh / s.P;
-  g.nw = s.Ww / s.P;
-  g.nb = s.T * g.nh * g.nw;
+  g.nt = s.T / g.pt;
+  g.nh = s.Hh / g.ph;
+  g.nw = s.Ww / g.pw;
+  g.nb = g.nt * g.nh * g.nw;
   g.S = s.T * s.Hh * s.Ww;
-  const int pairs_t = (s.T / 2) * g.nh * g.nw;
-  g.ntile = pairs_t + ((s.T & 1) ? g.nh * ((g.nw + 1) / 2) : 0);
+  const int pairs_t = (g.nt / 2) * g.nh * g.nw;
+  g.ntile = pairs_t + ((g.nt & 1) ? g.nh * ((g.nw + 1) / 2) : 0);
   return g;
 }
 
-// Block b (fractal block order) -> frame t, patch row hp, patch column wp.
+// Block b (fractal block order) -> block coordinates (t, hp, wp) along
+// (time, rows, columns), in units of the block shape.
 SA_HD void block_coords(const Geometry& g, int b, int& t, int& hp, int& wp) {
   const int per_frame = g.nh * g.nw;
   t = b / per_frame;
@@ -46,11 +58,11 @@ SA_HD void block_coords(const Geometry& g, int b, int& t, int& hp, int& wp) {
 }
 
 // Query tile -> the two q-blocks it holds (qb = -1 when alone). Pairs are
-// the same patch in frames (2i, 2i+1); an odd last frame pairs neighbouring
-// patch columns.
+// the same patch in block frames (2i, 2i+1); an odd last block frame pairs
+// neighbouring patch columns.
 SA_HD void tile_blocks(const Geometry& g, int tile, int& qa, int& qb) {
   const int per_frame = g.nh * g.nw;
-  const int pairs_t = (g.T / 2) * per_frame;
+  const int pairs_t = (g.nt / 2) * per_frame;
   if (tile < pairs_t) {
     const int tp = tile / per_frame;
     qa = 2 * tp * per_frame + (tile - tp * per_frame);
@@ -59,7 +71,7 @@ SA_HD void tile_blocks(const Geometry& g, int tile, int& qa, int& qb) {
     const int i = tile - pairs_t;
     const int half = (g.nw + 1) / 2;
     const int hp = i / half, wq = i - hp * half;
-    qa = (g.T - 1) * per_frame + hp * g.nw + 2 * wq;
+    qa = (g.nt - 1) * per_frame + hp * g.nw + 2 * wq;
     qb = (2 * wq + 1 < g.nw) ? qa + 1 : -1;
   }
 }

@@ -59,6 +59,12 @@ class Workload:
     seed: int = 0
     sigma: float = SIGMA
     field_var: float = FIELD_VAR
+    tile: Optional[Tuple[int, int, int]] = None  # block shape (pt, ph, pw); None = (1, P, P)
+
+    @property
+    def block(self):
+        """The block shape as the oracle takes it: the tile, or the patch edge P."""
+        return self.tile if self.tile is not None else self.P
 
     @property
     def S(self) -> int:
@@ -81,6 +87,7 @@ class Workload:
             "grid": [self.T, self.Hh, self.Ww], "tokens": self.S, "P": self.P,
             "N": self.N, "thr": self.thr, "sta": list(self.sta),
             "pos_scale": self.scale, "seed": self.seed,
+            "tile": list(self.tile) if self.tile is not None else [1, self.P, self.P],
         }
 
 
@@ -115,7 +122,14 @@ def sweep(k: int) -> Workload:
 
 N_SWEEP = len(SWEEP_THR) * len(SWEEP_STA) * len(SWEEP_SCALE)
 
-WORKLOADS = {w.name: w for w in (TINY, W8K, WAN, HUNYUAN)}
+# The same inputs with three-dimensional blocks (head-aware tile shapes):
+# pt frames x ph rows x pw columns, pt*ph*pw = 64.
+W8K_T248 = dataclasses.replace(W8K, name="8k_1x12x8192x128_sta3_tile2x4x8", tile=(2, 4, 8))
+W8K_T444 = dataclasses.replace(W8K, name="8k_1x12x8192x128_sta3_tile4x4x4", tile=(4, 4, 4))
+HUNYUAN_T1416 = dataclasses.replace(HUNYUAN, name="hunyuan_1x24x126720x128_tile1x4x16",
+                                    tile=(1, 4, 16))
+
+WORKLOADS = {w.name: w for w in (TINY, W8K, WAN, HUNYUAN, W8K_T248, W8K_T444, HUNYUAN_T1416)}
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:

@@ -52,6 +52,14 @@ typedef struct sa_desc {
   int sta_t, sta_h, sta_w; /* odd STA window in blocks, or 0,0,0 = no STA */
   int out_fp32;      /* 0: output bf16; 1: output fp32 (same layout) */
   int debug_flags;   /* 0 in normal use; SA_DEBUG_* bits for tests */
+  int pt, ph, pw;    /* block shape: 0,0,0 = the P x P patch of one frame
+                        (1, P, P); otherwise a three-dimensional tile of pt
+                        frames x ph rows x pw columns with pt*ph*pw == N, T % pt,
+                        Hh % ph and Ww % pw all 0 (the head-aware tiling of
+                        "Veda: Video Generation with Efficient Sparse
+                        Attention", section 2.2); P is then not used. Block
+                        coordinates, tile pairing and the STA window are in
+                        units of these tiles. */
 } sa_desc;
 
 /* Test-only: the attention kernel's loader never signals its first K/V
@@ -64,7 +72,8 @@ typedef enum sa_status {
   SA_ERR_INVALID_ARG = 1,     /* NULL pointer, non-positive size, thr out of
                                  range, even STA window, misaligned pointer */
   SA_ERR_UNSUPPORTED = 2,     /* valid but not implemented: d not in {64,128},
-                                 N != P*P, N != 64, grid not divisible by P */
+                                 N != 64, block shape not N tokens, grid not
+                                 divisible by the block shape */
   SA_ERR_WORKSPACE = 3,       /* workspace smaller than
                                  sparse_attn_workspace_size() */
   SA_ERR_CUDA = 4,            /* a CUDA runtime call or launch failed */
@@ -77,7 +86,9 @@ sa_status sparse_attn_workspace_size(const sa_desc* desc, size_t* bytes);
 /* Builds the block mask M = M_nabla OR M_STA for every (batch, head):
  *   1. fractal flattening: block b of a head is the P x P patch (hp, wp) of
  *      frame t, b = (t*(Hh/P) + hp)*(Ww/P) + wp, tokens row-major inside it
- *      (NABLA, Metodologia 1);
+ *      (NABLA, Metodologia 1); with a tile shape (pt, ph, pw) block
+ *      b = (tb*(Hh/ph) + hb)*(Ww/pw) + wb holds frames tb*pt.., rows hb*ph..,
+ *      columns wb*pw.., tokens in (t, h, w) row-major order inside it;
  *   2. Qbar, Kbar = mean of the N tokens of each block, fp32 (Metodologia 2,
  *      "Sottocampionamento");
  *   3. A = row softmax(Qbar Kbar^T / sqrt(d)) (Metodologia 2, "Attenzione

@@ -95,3 +95,45 @@ def test_tile_pairing_covers_every_block_once(T, Hh, Ww):
     assert sorted(seen) == list(range(nb))
     with pytest.raises(api.SparseAttnError):
         api.tile_blocks(d, ntile)
+
+
+def test_tile_shape_validation():
+    base = dict(B=1, H=2, T=8, Hh=32, Ww=32, d=128, thr=0.1)
+    cases = [
+        ((2, 4, 8), api.SA_OK),
+        ((4, 4, 4), api.SA_OK),
+        ((1, 8, 8), api.SA_OK),          # the square patch, given as a tile
+        ((2, 4, 4), api.SA_ERR_UNSUPPORTED),   # 32 tokens, not N = 64
+        ((3, 4, 8), api.SA_ERR_UNSUPPORTED),   # 96 tokens
+        ((16, 2, 2), api.SA_ERR_UNSUPPORTED),  # T = 8 not divisible by 16
+        ((1, 1, 64), api.SA_ERR_UNSUPPORTED),  # Ww = 32 not divisible by 64
+        ((0, 8, 8), api.SA_ERR_INVALID_ARG),
+        ((-2, -4, 8), api.SA_ERR_INVALID_ARG),
+    ]
+    for tile, expect in cases:
+        n = ctypes.c_size_t()
+        st = api.lib().sparse_attn_workspace_size(ctypes.byref(api.make_desc(**base, tile=tile)),
+                                                  ctypes.byref(n))
+        assert st == expect, (tile, st)
+    # with a tile the patch edge is not used
+    d = api.make_desc(**base, tile=(2, 4, 8), P=0)
+    assert api.workspace_size(d) > 0
+
+
+@pytest.mark.parametrize("T,Hh,Ww,tile", [(8, 32, 32, (2, 4, 8)), (8, 32, 32, (4, 4, 4)),
+                                         (33, 48, 80, (1, 4, 16)), (6, 16, 32, (2, 2, 16))])
+def test_tile_pairing_covers_every_block_once_3d(T, Hh, Ww, tile):
+    pt, ph, pw = tile
+    d = api.make_desc(1, 1, T, Hh, Ww, 128, 0.1, tile=tile)
+    nt, nh, nw = T // pt, Hh // ph, Ww // pw
+    nb = nt * nh * nw
+    seen = []
+    ntile = (nt // 2) * nh * nw + (nt % 2) * nh * ((nw + 1) // 2)
+    for i in range(ntile):
+        qa, qb = api.tile_blocks(d, i)
+        seen.append(qa)
+        if qb >= 0:
+            seen.append(qb)
+            ta, tb = qa // (nh * nw), qb // (nh * nw)
+            assert (tb == ta + 1 and qb - qa == nh * nw) or (ta == tb == nt - 1 and qb == qa + 1)
+    assert sorted(seen) == list(range(nb))

@@ -48,7 +48,7 @@ def run(w, out_fp32=False, debug_flags=0, inputs=None):
 def oracle_mask(w, heads=None):
     q, k, _ = host_inputs(w)
     sel = range(w.BH) if heads is None else heads
-    return oracle.nabla_mask(q[list(sel)], k[list(sel)], w.T, w.Hh, w.Ww, w.P, w.N, w.thr, w.sta)
+    return oracle.nabla_mask(q[list(sel)], k[list(sel)], w.T, w.Hh, w.Ww, w.block, w.N, w.thr, w.sta)
 
 
 def check_mask(w, gm, heads=None):
@@ -63,7 +63,7 @@ def check_mask(w, gm, heads=None):
 
 def check_out_full(w, out, gm, bf16_out=True):
     q, k, v = host_inputs(w)
-    ref, _ = oracle.nabla_attention(q, k, v, w.T, w.Hh, w.Ww, w.P, w.N, w.thr, w.sta, mask=gm)
+    ref, _ = oracle.nabla_attention(q, k, v, w.T, w.Hh, w.Ww, w.block, w.N, w.thr, w.sta, mask=gm)
     r = parity.out_check(out, ref, bf16_out)
     assert r["ok"], r
     return r
@@ -75,7 +75,7 @@ def check_out_sampled(w, out, gm, heads, n_tok=96, seed=0, bf16_out=True):
     got, refs = [], []
     for bh in heads:
         toks = rng.choice(w.S, size=n_tok, replace=False)
-        refs.append(oracle.attention_head(q[bh], k[bh], v[bh], w.T, w.Hh, w.Ww, w.P, w.N, gm[bh],
+        refs.append(oracle.attention_head(q[bh], k[bh], v[bh], w.T, w.Hh, w.Ww, w.block, w.N, gm[bh],
                                           tokens=toks))
         got.append(out[bh][toks])
     r = parity.out_check(np.concatenate(got), np.concatenate(refs), bf16_out)
@@ -108,12 +108,69 @@ def test_permute_bit_exact():
     desc = api.desc_for(w)
     y = torch.empty_like(x)
     api.permute(desc, x, y)
-    perm = oracle.fractal_order(w.T, w.Hh, w.Ww, w.P)
+    perm = oracle.fractal_order(w.T, w.Hh, w.Ww, w.block)
     got = y.view(torch.int16).cpu().numpy().reshape(w.BH, w.S, w.d).view(np.uint16)
     assert np.array_equal(got, oracle.flatten(q, perm))
     z = torch.empty_like(x)
     api.permute(desc, y, z, inverse=True)
     assert torch.equal(z.view(torch.int16), x.view(torch.int16))
+
+
+# ---------------------------------------------------------------- 3-D tiles
+
+@pytest.mark.parametrize("wname", ["8k_1x12x8192x128_sta3_tile2x4x8",
+                                   "8k_1x12x8192x128_sta3_tile4x4x4"])
+@pytest.mark.parametrize("out_fp32", [False, True])
+def test_3d_tile_full(wname, out_fp32):
+    w = W.WORKLOADS[wname]
+    out, gm, *_ = run(w, out_fp32=out_fp32)
+    check_mask(w, gm)
+    check_out_full(w, out, gm, bf16_out=not out_fp32)
+
+
+@pytest.mark.parametrize("wname", ["8k_1x12x8192x128_sta3_tile2x4x8",
+                                   "8k_1x12x8192x128_sta3_tile4x4x4"])
+def test_3d_tile_permute_and_pool(wname):
+    w = W.WORKLOADS[wname]
+    q, k, _ = host_inputs(w)
+    x = to_dev(q, w)
+    desc = api.desc_for(w)
+    y = torch.empty_like(x)
+    api.permute(desc, x, y)
+    perm = oracle.fractal_order(w.T, w.Hh, w.Ww, w.block)
+    got = y.view(torch.int16).cpu().numpy().reshape(w.BH, w.S, w.d).view(np.uint16)
+    assert np.array_equal(got, oracle.flatten(q, perm))
+    z = torch.empty_like(x)
+    api.permute(desc, y, z, inverse=True)
+    assert torch.equal(z.view(torch.int16), x.view(torch.int16))
+    _, _, views, *_ = run(w)
+    for bh in (0, w.BH - 1):
+        for name, src in (("qbar", q), ("kbar", k)):
+            ref = oracle.pooled_head(src[bh], w.T, w.Hh, w.Ww, w.block, w.N)
+            got_p = views[name][bh].cpu().numpy().astype(np.float64)
+            assert np.abs(got_p - ref).max() <= 1e-6 * max(1.0, np.abs(ref).max())
+
+
+def test_3d_tile_union_lists():
+    w = W.W8K_T248
+    _, gm, views, desc, _ = run(w)
+    tc = views["tile_cnt"].cpu().numpy()
+    ti = views["tile_idx"].cpu().numpy()
+    pf = (w.Hh // w.tile[1]) * (w.Ww // w.tile[2])
+    for bh in (0, w.BH - 1):
+        for t in range(views["ntile"]):
+            qa, qb = api.tile_blocks(desc, t)
+            ma = gm[bh, qa]
+            mb = gm[bh, qb] if qb >= 0 else np.zeros_like(ma)
+            ent = ti[bh, t, :tc[bh, t]]
+            blocks = ent & 0xFFFF
+            assert sorted(blocks.tolist()) == np.nonzero(ma | mb)[0].tolist()
+            assert np.array_equal((ent >> 16) & 1, ma[blocks].astype(np.int32))
+            assert np.array_equal((ent >> 17) & 1, mb[blocks].astype(np.int32))
+            # temporal pairs lead: flagged entry b followed by b + one block frame
+            fl = np.nonzero((ent >> 18) & 1)[0]
+            for i in fl:
+                assert blocks[i + 1] == blocks[i] + pf
 
 
 def test_pooled_blocks_match_oracle():
@@ -122,7 +179,7 @@ def test_pooled_blocks_match_oracle():
     q, k, _ = host_inputs(w)
     for bh in (0, 5, w.BH - 1):
         for name, x in (("qbar", q), ("kbar", k)):
-            ref = oracle.pooled_head(x[bh], w.T, w.Hh, w.Ww, w.P, w.N)
+            ref = oracle.pooled_head(x[bh], w.T, w.Hh, w.Ww, w.block, w.N)
             got = views[name][bh].cpu().numpy().astype(np.float64)
             assert np.abs(got - ref).max() <= 1e-6 * max(1.0, np.abs(ref).max())
 
