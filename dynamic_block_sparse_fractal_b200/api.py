@@ -27,6 +27,8 @@ SYMBOLS = (
     "sparse_attn_workspace_size", "sparse_attn_plan", "sparse_attn_fwd",
     "sparse_attn_permute", "sparse_attn_get_mask", "sparse_attn_tile_blocks",
     "sparse_attn_check", "sparse_attn_forward_noalloc", "sparse_attn_status_string",
+    "sparse_attn_workspace_size_heads", "sparse_attn_plan_heads", "sparse_attn_fwd_heads",
+    "sparse_attn_check_heads", "sparse_attn_heads_run",
 )
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -74,6 +76,13 @@ def lib() -> ctypes.CDLL:
         L.sparse_attn_tile_blocks.argtypes = [dp, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)]
         L.sparse_attn_check.argtypes = [dp, vp, sz, vp]
         L.sparse_attn_forward_noalloc.argtypes = [dp, vp, vp, vp, vp, vp]
+        ip = ctypes.POINTER(i32)
+        L.sparse_attn_workspace_size_heads.argtypes = [dp, ip, ctypes.POINTER(sz)]
+        L.sparse_attn_plan_heads.argtypes = [dp, ip, vp, vp, vp, sz, vp]
+        L.sparse_attn_fwd_heads.argtypes = [dp, ip, vp, vp, vp, vp, sz, vp, vp]
+        L.sparse_attn_check_heads.argtypes = [dp, ip, vp, sz, vp]
+        L.sparse_attn_heads_run.argtypes = [dp, ip, i32, dp, ip, ctypes.POINTER(sz),
+                                            ctypes.POINTER(sz)]
         L.sparse_attn_status_string.argtypes = [i32]
         L.sparse_attn_status_string.restype = ctypes.c_char_p
         for name in SYMBOLS:
@@ -209,6 +218,59 @@ def get_mask(desc: SaDesc, workspace: torch.Tensor) -> dict:
         "tile_cnt": view(v.tile_cnt, BH * nt, torch.int32, (BH, nt)),
         "tile_idx": view(v.tile_idx, BH * nt * nb, torch.int32, (BH, nt, nb)),
     }
+
+
+# ---- per-head block shapes (head-aware tiling) -------------------------------
+
+def _tiles_array(tiles):
+    flat = [int(v) for t in tiles for v in t]
+    return (ctypes.c_int * len(flat))(*flat)
+
+
+def workspace_size_heads(desc: SaDesc, tiles) -> int:
+    n = ctypes.c_size_t(0)
+    _ok(lib().sparse_attn_workspace_size_heads(ctypes.byref(desc), _tiles_array(tiles),
+                                               ctypes.byref(n)), "workspace_size_heads")
+    return n.value
+
+
+def plan_heads(desc: SaDesc, tiles, q, k, workspace, stream=None) -> None:
+    _check_qkv(desc, q, k)
+    _ok(lib().sparse_attn_plan_heads(ctypes.byref(desc), _tiles_array(tiles), _ptr(q), _ptr(k),
+                                     _ptr(workspace), workspace.numel(), _stream(stream)),
+        "plan_heads")
+
+
+def fwd_heads(desc: SaDesc, tiles, q, k, v, workspace, out, stream=None):
+    _check_qkv(desc, q, k, v)
+    want = torch.float32 if desc.out_fp32 else torch.bfloat16
+    if out.dtype != want or out.shape != q.shape or not out.is_contiguous():
+        raise ValueError(f"out must be a contiguous {want} tensor shaped like q")
+    _ok(lib().sparse_attn_fwd_heads(ctypes.byref(desc), _tiles_array(tiles), _ptr(q), _ptr(k),
+                                    _ptr(v), _ptr(workspace), workspace.numel(), _ptr(out),
+                                    _stream(stream)), "fwd_heads")
+    return out
+
+
+def check_heads(desc: SaDesc, tiles, workspace, stream=None) -> int:
+    return lib().sparse_attn_check_heads(ctypes.byref(desc), _tiles_array(tiles),
+                                         _ptr(workspace), workspace.numel(), _stream(stream))
+
+
+def heads_runs(desc: SaDesc, tiles):
+    """[(sub_desc, head0, ws_offset, ws_bytes)] for the runs of equal shapes."""
+    out, i = [], 0
+    arr = _tiles_array(tiles)
+    while True:
+        sub, h0 = SaDesc(), ctypes.c_int(0)
+        off, nbytes = ctypes.c_size_t(0), ctypes.c_size_t(0)
+        st = lib().sparse_attn_heads_run(ctypes.byref(desc), arr, i, ctypes.byref(sub),
+                                         ctypes.byref(h0), ctypes.byref(off), ctypes.byref(nbytes))
+        if st == SA_ERR_INVALID_ARG and i > 0:
+            return out
+        _ok(st, "heads_run")
+        out.append((sub, h0.value, off.value, nbytes.value))
+        i += 1
 
 
 class NablaAttention:

@@ -191,6 +191,43 @@ sa_status sparse_attn_forward_noalloc(const sa_desc* desc, const void* q,
                                       const void* k, const void* v, void* out,
                                       void* stream);
 
+/* ---- Per-head block shapes ------------------------------------------------
+ * The head-aware tiling of "Veda: Video Generation with Efficient Sparse
+ * Attention" (section 2.2, "Tiling Consapevole delle Teste"): each head may
+ * use its own block shape. tiles is a HOST array of B*H triples
+ * (pt, ph, pw), in (batch, head) order; each must satisfy the single-shape
+ * rules of sa_desc (pt*ph*pw == N, the grid divisible by it; 0,0,0 = the
+ * P x P patch). desc->pt/ph/pw are ignored. Consecutive heads with equal
+ * triples form a run, which is planned and run as one problem with H = run
+ * length on its slice of q, k, v, out (a head's [S, d] rows are contiguous)
+ * and its own 256-byte-aligned slice of the workspace, so results equal
+ * separate single-shape calls head by head. Errors: those of the
+ * single-shape calls, for the first run that fails; a NULL tiles is
+ * SA_ERR_INVALID_ARG. */
+
+/* Workspace bytes for all runs together. */
+sa_status sparse_attn_workspace_size_heads(const sa_desc* desc, const int* tiles, size_t* bytes);
+
+/* sparse_attn_plan for every run (q, k: the full [B, H, S, d] tensors). */
+sa_status sparse_attn_plan_heads(const sa_desc* desc, const int* tiles, const void* q,
+                                 const void* k, void* workspace, size_t ws_bytes, void* stream);
+
+/* sparse_attn_fwd for every run; out: the full [B, H, S, d] output. */
+sa_status sparse_attn_fwd_heads(const sa_desc* desc, const int* tiles, const void* q,
+                                const void* k, const void* v, const void* workspace,
+                                size_t ws_bytes, void* out, void* stream);
+
+/* sparse_attn_check over every run's status word (synchronises stream). */
+sa_status sparse_attn_check_heads(const sa_desc* desc, const int* tiles, const void* workspace,
+                                  size_t ws_bytes, void* stream);
+
+/* Host-only: run number `run` (0-based) as a single-shape problem: its
+ * descriptor (*sub, B = 1, H = run length), first flattened head (*head0)
+ * and workspace slice (*ws_offset, *ws_bytes), e.g. for sparse_attn_get_mask
+ * on that slice. SA_ERR_INVALID_ARG when run is past the last run. */
+sa_status sparse_attn_heads_run(const sa_desc* desc, const int* tiles, int run, sa_desc* sub,
+                                int* head0, size_t* ws_offset, size_t* ws_bytes);
+
 #ifdef __cplusplus
 }
 #endif

@@ -137,3 +137,29 @@ def test_tile_pairing_covers_every_block_once_3d(T, Hh, Ww, tile):
             ta, tb = qa // (nh * nw), qb // (nh * nw)
             assert (tb == ta + 1 and qb - qa == nh * nw) or (ta == tb == nt - 1 and qb == qa + 1)
     assert sorted(seen) == list(range(nb))
+
+
+def test_per_head_shapes_split_into_runs():
+    w = W.W8K  # 12 heads on an 8 x 32 x 32 grid
+    d = api.desc_for(w)
+    tiles = [(1, 8, 8)] * 4 + [(2, 4, 8)] * 4 + [(4, 4, 4)] * 2 + [(2, 4, 8)] * 2
+    runs = api.heads_runs(d, tiles)
+    assert [(r[0].H, r[1]) for r in runs] == [(4, 0), (4, 4), (2, 8), (2, 10)]
+    assert [(r[0].pt, r[0].ph, r[0].pw) for r in runs] == [(1, 8, 8), (2, 4, 8), (4, 4, 4),
+                                                           (2, 4, 8)]
+    total = api.workspace_size_heads(d, tiles)
+    off = 0
+    for sub, _, ws_off, ws_bytes in runs:
+        assert ws_off == off and ws_off % 256 == 0
+        assert ws_bytes == api.workspace_size(sub)
+        off = (ws_off + ws_bytes + 255) // 256 * 256
+    assert total == off
+    # one shape for every head: a single run with the whole problem
+    one = api.heads_runs(d, [(2, 4, 8)] * 12)
+    assert len(one) == 1 and one[0][0].H == 12
+    # a bad shape in one head is that run's error; no tiles is an argument error
+    with pytest.raises(api.SparseAttnError):
+        api.workspace_size_heads(d, [(1, 8, 8)] * 11 + [(3, 4, 8)])
+    n = ctypes.c_size_t()
+    assert api.lib().sparse_attn_workspace_size_heads(ctypes.byref(d), None, ctypes.byref(n)) == \
+        api.SA_ERR_INVALID_ARG

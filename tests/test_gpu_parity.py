@@ -313,3 +313,29 @@ def test_sweep_all_variants_small_grid(k):
     out, gm, *_ = run(w)
     check_mask(w, gm)
     check_out_full(w, out, gm)
+
+
+def test_per_head_shapes_match_oracle_head_by_head():
+    w = W.W8K
+    tiles = [(1, 8, 8)] * 4 + [(2, 4, 8)] * 4 + [(4, 4, 4)] * 2 + [(2, 4, 8)] * 2
+    q, k, v = host_inputs(w)
+    qd, kd, vd = to_dev(q, w), to_dev(k, w), to_dev(v, w)
+    desc = api.desc_for(w)
+    ws = torch.empty(api.workspace_size_heads(desc, tiles), dtype=torch.uint8, device="cuda")
+    api.plan_heads(desc, tiles, qd, kd, ws)
+    out = torch.empty_like(qd)
+    api.fwd_heads(desc, tiles, qd, kd, vd, ws, out)
+    assert api.check_heads(desc, tiles, ws) == api.SA_OK
+    out_np = out.float().cpu().numpy().reshape(w.BH, w.S, w.d)
+    for sub, h0, off, nbytes in api.heads_runs(desc, tiles):
+        views = api.get_mask(sub, ws[off:off + nbytes])
+        gm = parity.lists_to_mask(views["cnt"].cpu().numpy(), views["idx"].cpu().numpy())
+        heads = list(range(h0, h0 + sub.H))
+        tile = (sub.pt, sub.ph, sub.pw)
+        M, Mn, A = oracle.nabla_mask(q[heads], k[heads], w.T, w.Hh, w.Ww, tile, w.N, w.thr, w.sta)
+        r = parity.compare_masks(gm, M, Mn, A, w.thr)
+        assert r["bad"] == 0 and r["sta_missing"] == 0, (tile, r)
+        ref, _ = oracle.nabla_attention(q[heads], k[heads], v[heads], w.T, w.Hh, w.Ww, tile, w.N,
+                                        w.thr, w.sta, mask=gm)
+        res = parity.out_check(out_np[heads], ref, True)
+        assert res["ok"], (tile, res)
