@@ -39,18 +39,26 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
 #pragma unroll
   for (int i = 0; i < kPerLane; ++i) acc[i] = 0.f;
   // token r of the block: frame t*pt + (r >> (lph + lpw)), row hp*ph +
-  // ((r >> lpw) & (ph - 1)), column wp*pw + (r & (pw - 1))
+  // ((r >> lpw) & (ph - 1)), column wp*pw + (r & (pw - 1)); the 8 x 8 patch
+  // of one frame (the default block) takes a loop with constant addressing
   const size_t base_tok = (size_t(t) * g.pt * g.Hh + size_t(hp) * g.ph) * g.Ww + size_t(wp) * g.pw;
+  const bool patch8 = g.pt == 1 && g.ph == 8 && g.pw == 8;
 #pragma unroll 2
   for (int r0 = 0; r0 < 64; r0 += 8) {
     float2 raw[8];
+    const size_t run0 = patch8 ? base_tok + size_t(r0 >> 3) * g.Ww : 0;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-      const int r = r0 + u;
-      const int run = r >> g.lpw, wi = r & (g.pw - 1);
-      const int ti = run >> g.lph, hi = run & (g.ph - 1);
-      const __nv_bfloat16* p =
-          src + (base_tok + (size_t(ti) * g.Hh + hi) * g.Ww + wi) * D;
+      size_t tok;
+      if (patch8) {
+        tok = run0 + u;
+      } else {
+        const int r = r0 + u;
+        const int run = r >> g.lpw, wi = r & (g.pw - 1);
+        const int ti = run >> g.lph, hi = run & (g.ph - 1);
+        tok = base_tok + (size_t(ti) * g.Hh + hi) * g.Ww + wi;
+      }
+      const __nv_bfloat16* p = src + tok * D;
       if constexpr (kPerLane == 4) {
         raw[u] = __ldg(reinterpret_cast<const float2*>(p));
       } else {
