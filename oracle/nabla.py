@@ -242,3 +242,32 @@ def nabla_attention(q, k, v, T, Hh, Ww, P, N, thr, sta, mask=None):
     out = np.stack([attention_head(q[bh], k[bh], v[bh], T, Hh, Ww, P, N, mask[bh])
                     for bh in range(q.shape[0])])
     return out, mask
+
+
+# --- Block max-pooled attention map (quality signal for a block mask) --------
+# The reference target of the page "Veda: Video Generation with Efficient
+# Sparse Attention", section 2.1 ("Costruzione dell'Obiettivo"): the full
+# attention matrix, max-pooled over the (query block, key block) regions.
+
+def block_heatmap(q, k, T, Hh, Ww, P, N):
+    """H[qb, kb] = max over the N x N block of the full softmax attention
+    probabilities (all keys, no mask) of one head, blocks in fractal order.
+
+    q, k: natural-order [S, d]. Returns float64 [nb, nb].
+    """
+    perm = fractal_order(T, Hh, Ww, P)
+    qp, kp = flatten(_as_f64(q), perm), flatten(_as_f64(k), perm)
+    S, d = qp.shape
+    s = qp @ kp.T / np.sqrt(d)
+    p = np.exp(s - s.max(axis=-1, keepdims=True))
+    p /= p.sum(axis=-1, keepdims=True)
+    nb = S // N
+    return p.reshape(nb, N, nb, N).max(axis=(1, 3))
+
+
+def heat_recall(H, M):
+    """Per q-block row, the share of the row's max-pooled attention (sum of
+    H over its key blocks) that the kept blocks of mask M cover; the mean
+    over rows. 1.0 = the mask keeps every block that carries attention."""
+    H = np.asarray(H, dtype=np.float64)
+    return float(np.mean((H * M).sum(axis=-1) / H.sum(axis=-1)))

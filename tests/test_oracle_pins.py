@@ -482,3 +482,47 @@ def test_planted_mistake_is_caught(name, mutant, area, golden_dir, monkeypatch):
         except AssertionError:
             caught += 1
     assert caught >= 1, f"no pin caught the planted mistake {mutant.__name__}"
+
+
+# --- block max-pooled attention map -------------------------------------------
+
+def test_block_heatmap_bruteforce_token_by_token():
+    # Tiny problem: compute every probability by an explicit loop over tokens
+    # (exp of the scaled dot product over the sum over all keys), then the
+    # block max by looping over the positions of each block.
+    rng = np.random.default_rng(29)
+    T, Hh, Ww, P, N = 2, 8, 8, 8, 64
+    S, d = T * Hh * Ww, 4
+    q, k = rng.standard_normal((S, d)), rng.standard_normal((S, d))
+    H = oracle.block_heatmap(q, k, T, Hh, Ww, P, N)
+    perm = oracle.fractal_order(T, Hh, Ww, P)  # position -> natural token
+    nb = S // N
+    expect = np.zeros((nb, nb))
+    for i in range(S):
+        s = np.array([math.exp(float(q[i] @ k[j]) / math.sqrt(d)) for j in range(S)])
+        prob = s / s.sum()
+        pos = int(np.nonzero(perm == i)[0][0])
+        for j in range(S):
+            pj = int(np.nonzero(perm == j)[0][0])
+            expect[pos // N, pj // N] = max(expect[pos // N, pj // N], prob[j])
+    assert np.abs(H - expect).max() < 1e-12
+
+
+def test_block_heatmap_closed_forms_and_bounds():
+    T, Hh, Ww, P, N = 2, 16, 16, 8, 64
+    S = T * Hh * Ww
+    zero = np.zeros((S, 8))
+    H = oracle.block_heatmap(zero, np.random.default_rng(1).standard_normal((S, 8)),
+                             T, Hh, Ww, P, N)
+    assert np.allclose(H, 1.0 / S, rtol=0, atol=1e-15)  # zero queries attend uniformly
+    rng = np.random.default_rng(31)
+    q, k = rng.standard_normal((S, 8)) * 2, rng.standard_normal((S, 8)) * 2
+    H = oracle.block_heatmap(q, k, T, Hh, Ww, P, N)
+    assert (H <= 1).all() and (H > 0).all()
+    # a row's probabilities sum to 1 over nb blocks of N keys: the block
+    # maxima of one q-block sum to at least 1/N
+    assert (H.sum(axis=1) >= 1.0 / N - 1e-12).all()
+    M = np.zeros(H.shape, dtype=bool)
+    assert oracle.heat_recall(H, ~M) == 1.0 and oracle.heat_recall(H, M) == 0.0
+    top = H >= np.sort(H, axis=1)[:, -2:-1]  # two largest per row
+    assert 0.0 < oracle.heat_recall(H, top) < 1.0
