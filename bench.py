@@ -280,6 +280,9 @@ def run_ours(args, w, rank, world):
     if st != api.SA_OK:
         raise SystemExit(f"device status after e2e: {api.status_string(st)}")
 
+    heatmap = None if args.no_heatmap else measure_heatmap(api, desc, w, q, k, ws, views, dev,
+                                                             stream)
+
     peaks, src = load_peaks()
     ms_step = total_ms / args.steps
     fwd_avg = statistics.mean(fwd_ms)
@@ -311,10 +314,44 @@ def run_ours(args, w, rank, world):
         "gpu_launches": 6 * args.steps,  # pool, logits, select, union, tile order, attention
         "clocks": clocks.summary(),
     }
+    if heatmap is not None:
+        heatmap["frac"] = round(heatmap["tensor_tflops"] / peak, 4)
+        line["heatmap"] = heatmap
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
     return line
+
+
+def measure_heatmap(api, desc, w, q, k, ws, views, dev, stream, reps=3):
+    """Times the exact block max-pooled attention map (one launch of the heat
+    kernel after its zeroing) outside the step, and reports the recall of the
+    planned NABLA mask against it: per q-block, the share of the block maxima
+    that the kept blocks cover, averaged over q-blocks and heads."""
+    import torch
+    heat = torch.empty((w.BH, w.nb, w.nb), dtype=torch.float32, device=dev)
+    api.block_heatmap(desc, q, k, ws, heat)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(reps):
+        api.block_heatmap(desc, q, k, ws, heat)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / reps
+    st = api.check(desc, ws)
+    if st != api.SA_OK:
+        raise SystemExit(f"device status after the heat map: {api.status_string(st)}")
+    cnt = views["cnt"].long()
+    idx = views["idx"].long().clamp_(0, w.nb - 1)
+    kept = torch.arange(w.nb, device=dev).view(1, 1, -1) < cnt.unsqueeze(-1)
+    covered = (torch.gather(heat, 2, idx) * kept).sum(-1)
+    recall = float((covered / heat.sum(-1)).mean().item())
+    qk_flops = 2.0 * w.S * w.S * w.d * w.BH  # one dense Q K^T
+    return {"kernel": "sa::heat_kernel<%d>" % w.d, "ms": round(ms, 3),
+            "tensor_tflops": round(2 * qk_flops / (ms * 1e-3) / 1e12, 2),
+            "note": "two dense Q K^T passes (row log-sum-exp, then block maxima)",
+            "mask_recall": round(recall, 4)}
 
 
 def oracle_sample(w, budget_s=20.0, seed=0):
@@ -385,6 +422,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-heatmap", action="store_true",
+                    help="skip the block max-pooled attention map measurement")
     ap.add_argument("--heads", type=int, default=None,
                     help="run the workload's grid with this many heads (small ncu captures); "
                          "the line's config then names the changed workload")

@@ -28,7 +28,7 @@ SYMBOLS = (
     "sparse_attn_permute", "sparse_attn_get_mask", "sparse_attn_tile_blocks",
     "sparse_attn_check", "sparse_attn_forward_noalloc", "sparse_attn_status_string",
     "sparse_attn_workspace_size_heads", "sparse_attn_plan_heads", "sparse_attn_fwd_heads",
-    "sparse_attn_check_heads", "sparse_attn_heads_run",
+    "sparse_attn_check_heads", "sparse_attn_heads_run", "sparse_attn_block_heatmap",
 )
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -187,6 +187,23 @@ def check(desc: SaDesc, workspace: torch.Tensor, stream=None) -> int:
     """Synchronises the stream; returns the status (SA_OK or an error code)."""
     return lib().sparse_attn_check(ctypes.byref(desc), _ptr(workspace), workspace.numel(),
                                    _stream(stream))
+
+
+def block_heatmap(desc: SaDesc, q: torch.Tensor, k: torch.Tensor, workspace: torch.Tensor,
+                  heat: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Exact block max-pooled full-attention map [B*H, nb, nb] (fp32, fractal
+    block order); see include/sparse_attn.h."""
+    _check_qkv(desc, q, k)
+    nb = desc.T * desc.Hh * desc.Ww // desc.N
+    shape = (desc.B * desc.H, nb, nb)
+    if heat is None:
+        heat = torch.empty(shape, dtype=torch.float32, device=q.device)
+    if heat.dtype != torch.float32 or tuple(heat.shape) != shape or not heat.is_contiguous():
+        raise ValueError(f"heat must be a contiguous float32 tensor of shape {shape}")
+    _ok(lib().sparse_attn_block_heatmap(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(workspace),
+                                        workspace.numel(), _ptr(heat), _stream(stream)),
+        "block_heatmap")
+    return heat
 
 
 def tile_blocks(desc: SaDesc, tile: int) -> Tuple[int, int]:

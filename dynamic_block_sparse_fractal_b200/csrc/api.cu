@@ -162,6 +162,30 @@ sa_status sparse_attn_fwd(const sa_desc* desc, const void* q, const void* k, con
   return cuda_status(launch_attn(a, g, static_cast<cudaStream_t>(stream)));
 }
 
+sa_status sparse_attn_block_heatmap(const sa_desc* desc, const void* q, const void* k,
+                                   void* workspace, size_t ws_bytes, float* heat, void* stream) {
+  sa_status st = validate(desc);
+  if (st != SA_OK) return st;
+  if (q == nullptr || k == nullptr || heat == nullptr || !aligned(q, 16) || !aligned(k, 16) ||
+      !aligned(heat, 4))
+    return SA_ERR_INVALID_ARG;
+  const Geometry g = make_geometry(*desc);
+  st = check_ws(g, workspace, ws_bytes);
+  if (st != SA_OK) return st;
+  const WsLayout w = make_ws_layout(g);
+  HeatArgs a;
+  std::memset(&a, 0, sizeof(a));
+  if (!encode_tile_map(&a.map_q, q, g.BH, g.T, g.Hh, g.Ww, g.d, g.pt, g.ph, g.pw) ||
+      !encode_tile_map(&a.map_k, k, g.BH, g.T, g.Hh, g.Ww, g.d, g.pt, g.ph, g.pw))
+    return SA_ERR_CUDA;
+  a.heat = heat;
+  a.status = at<uint32_t>(workspace, w.status);
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)g.d));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(a.status, 0, sizeof(uint32_t), s) != cudaSuccess) return SA_ERR_CUDA;
+  return cuda_status(launch_heat(a, g, s));
+}
+
 sa_status sparse_attn_permute(const sa_desc* desc, const void* x, void* y, int inverse,
                               void* stream) {
   const sa_status st = validate(desc);

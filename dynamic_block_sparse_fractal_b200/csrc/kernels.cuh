@@ -59,4 +59,14 @@ struct AttnArgs {
 };
 cudaError_t launch_attn(const AttnArgs& a, const Geometry& g, cudaStream_t stream);
 
+// Exact block max-pooled attention map: heat[bh][qb][kb] = max over the
+// block pair of the full softmax probability (zeroes heat, then one launch).
+struct HeatArgs {
+  CUtensorMap map_q, map_k;  // 5-D patch maps, one block per box
+  float* heat;               // [BH][nb][nb], fractal block order
+  uint32_t* status;
+  float scale_log2;  // log2(e) / sqrt(d)
+};
+cudaError_t launch_heat(const HeatArgs& a, const Geometry& g, cudaStream_t stream);
+
 }  // namespace sa

@@ -228,6 +228,25 @@ sa_status sparse_attn_check_heads(const sa_desc* desc, const int* tiles, const v
 sa_status sparse_attn_heads_run(const sa_desc* desc, const int* tiles, int run, sa_desc* sub,
                                 int* head0, size_t* ws_offset, size_t* ws_bytes);
 
+/* ---- Block max-pooled attention map (mask diagnostics) -------------------
+ * "Veda: Video Generation with Efficient Sparse Attention", section 2.1
+ * ("Costruzione dell'Obiettivo"): the reference a block mask is judged
+ * against is the full, unmasked attention P = softmax(Q K^T / sqrt(d)) of a
+ * head, max-pooled over every N x N block:
+ *   heat[bh][i][j] = max over q in block i, k in block j of P[q][k],
+ * blocks in fractal block order (the order of sparse_attn_get_mask's ids).
+ * Computed exactly (dense, two passes over every key: the row log-sum-exp,
+ * then the block maxima), so it costs about twice a dense QK^T; meant for
+ * measuring a mask's recall, not for the attention path.
+ * q, k: as for sparse_attn_plan. workspace: as for sparse_attn_plan; only its
+ * status word is used: cleared on `stream` before the launch, so the next
+ * sparse_attn_check reports this call (a timed-out wait leaves heat
+ * incomplete); the planned lists are left as they are. heat: device fp32 [B*H][nb][nb], 4-byte aligned,
+ * owned by the caller, overwritten (zeroed first, on `stream`). */
+sa_status sparse_attn_block_heatmap(const sa_desc* desc, const void* q, const void* k,
+                                    void* workspace, size_t ws_bytes, float* heat,
+                                    void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -265,6 +265,24 @@ def block_heatmap(q, k, T, Hh, Ww, P, N):
     return p.reshape(nb, N, nb, N).max(axis=(1, 3))
 
 
+def block_heatmap_rows(q, k, T, Hh, Ww, P, N, qblocks):
+    """Rows ``qblocks`` (fractal block ids) of block_heatmap, computed from
+    the softmax rows of those blocks' queries only: float64 [len, nb]."""
+    perm = fractal_order(T, Hh, Ww, P)
+    qp, kp = flatten(_as_f64(q), perm), flatten(_as_f64(k), perm)
+    S, d = kp.shape
+    nb = S // N
+    out = np.empty((len(qblocks), nb))
+    for r, b in enumerate(qblocks):
+        if not 0 <= b < nb:
+            raise IndexError(f"q-block {b} outside [0, {nb})")
+        s = qp[b * N:(b + 1) * N] @ kp.T / np.sqrt(d)
+        p = np.exp(s - s.max(axis=-1, keepdims=True))
+        p /= p.sum(axis=-1, keepdims=True)
+        out[r] = p.reshape(N, nb, N).max(axis=(0, 2))
+    return out
+
+
 def heat_recall(H, M):
     """Per q-block row, the share of the row's max-pooled attention (sum of
     H over its key blocks) that the kept blocks of mask M cover; the mean

@@ -75,6 +75,13 @@ def test_entry_points_reject_before_launch():
     assert L.sparse_attn_check(ctypes.byref(d), FAKE, 0, None) == api.SA_ERR_WORKSPACE
     assert L.sparse_attn_get_mask(None, FAKE, need, ctypes.byref(v)) == api.SA_ERR_INVALID_ARG
     assert api.status_string(api.SA_ERR_DEVICE_TIMEOUT).startswith("a kernel")
+    st = L.sparse_attn_block_heatmap(ctypes.byref(d), FAKE, FAKE, FAKE, need, None, None)
+    assert st == api.SA_ERR_INVALID_ARG  # no heat buffer
+    st = L.sparse_attn_block_heatmap(ctypes.byref(d), FAKE, FAKE, FAKE, need,
+                                     ctypes.c_void_p(0x10000002), None)
+    assert st == api.SA_ERR_INVALID_ARG  # heat not 4-byte aligned
+    st = L.sparse_attn_block_heatmap(ctypes.byref(d), FAKE, FAKE, FAKE, need - 1, FAKE, None)
+    assert st == api.SA_ERR_WORKSPACE
 
 
 @pytest.mark.parametrize("T,Hh,Ww", [(4, 8, 8), (33, 48, 80), (21, 32, 56), (3, 8, 24), (1, 16, 8)])

@@ -506,6 +506,9 @@ def test_block_heatmap_bruteforce_token_by_token():
             pj = int(np.nonzero(perm == j)[0][0])
             expect[pos // N, pj // N] = max(expect[pos // N, pj // N], prob[j])
     assert np.abs(H - expect).max() < 1e-12
+    rows = [1, 0]  # the per-row form (only those q-blocks' softmax rows)
+    Hr = oracle.block_heatmap_rows(q, k, T, Hh, Ww, P, N, rows)
+    assert np.abs(Hr - expect[rows]).max() < 1e-12
 
 
 def test_block_heatmap_closed_forms_and_bounds():
