@@ -29,6 +29,7 @@ SYMBOLS = (
     "sparse_attn_check", "sparse_attn_forward_noalloc", "sparse_attn_status_string",
     "sparse_attn_workspace_size_heads", "sparse_attn_plan_heads", "sparse_attn_fwd_heads",
     "sparse_attn_check_heads", "sparse_attn_heads_run", "sparse_attn_block_heatmap",
+    "sparse_attn_block_heatmap_scratch_size",
 )
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -189,10 +190,19 @@ def check(desc: SaDesc, workspace: torch.Tensor, stream=None) -> int:
                                    _stream(stream))
 
 
+def heatmap_scratch_size(desc: SaDesc) -> int:
+    n = ctypes.c_size_t(0)
+    _ok(lib().sparse_attn_block_heatmap_scratch_size(ctypes.byref(desc), ctypes.byref(n)),
+        "block_heatmap_scratch_size")
+    return n.value
+
+
 def block_heatmap(desc: SaDesc, q: torch.Tensor, k: torch.Tensor, workspace: torch.Tensor,
-                  heat: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                  heat: Optional[torch.Tensor] = None, scratch: Optional[torch.Tensor] = None,
+                  stream=None) -> torch.Tensor:
     """Exact block max-pooled full-attention map [B*H, nb, nb] (fp32, fractal
-    block order); see include/sparse_attn.h."""
+    block order); see include/sparse_attn.h. ``scratch``: a uint8 device
+    buffer of heatmap_scratch_size(desc) bytes (allocated when None)."""
     _check_qkv(desc, q, k)
     nb = desc.T * desc.Hh * desc.Ww // desc.N
     shape = (desc.B * desc.H, nb, nb)
@@ -200,8 +210,12 @@ def block_heatmap(desc: SaDesc, q: torch.Tensor, k: torch.Tensor, workspace: tor
         heat = torch.empty(shape, dtype=torch.float32, device=q.device)
     if heat.dtype != torch.float32 or tuple(heat.shape) != shape or not heat.is_contiguous():
         raise ValueError(f"heat must be a contiguous float32 tensor of shape {shape}")
+    if scratch is None:
+        scratch = torch.empty(heatmap_scratch_size(desc), dtype=torch.uint8, device=q.device)
     _ok(lib().sparse_attn_block_heatmap(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(workspace),
-                                        workspace.numel(), _ptr(heat), _stream(stream)),
+                                        ctypes.c_size_t(workspace.numel()), _ptr(heat),
+                                        _ptr(scratch), ctypes.c_size_t(scratch.numel()),
+                                        _stream(stream)),
         "block_heatmap")
     return heat
 

@@ -162,16 +162,26 @@ sa_status sparse_attn_fwd(const sa_desc* desc, const void* q, const void* k, con
   return cuda_status(launch_attn(a, g, static_cast<cudaStream_t>(stream)));
 }
 
+sa_status sparse_attn_block_heatmap_scratch_size(const sa_desc* desc, size_t* bytes) {
+  const sa_status st = validate(desc);
+  if (st != SA_OK) return st;
+  if (bytes == nullptr) return SA_ERR_INVALID_ARG;
+  *bytes = heat_scratch_bytes(make_geometry(*desc));
+  return SA_OK;
+}
+
 sa_status sparse_attn_block_heatmap(const sa_desc* desc, const void* q, const void* k,
-                                   void* workspace, size_t ws_bytes, float* heat, void* stream) {
+                                    void* workspace, size_t ws_bytes, float* heat,
+                                    void* scratch, size_t scratch_bytes, void* stream) {
   sa_status st = validate(desc);
   if (st != SA_OK) return st;
-  if (q == nullptr || k == nullptr || heat == nullptr || !aligned(q, 16) || !aligned(k, 16) ||
-      !aligned(heat, 4))
+  if (q == nullptr || k == nullptr || heat == nullptr || scratch == nullptr ||
+      !aligned(q, 16) || !aligned(k, 16) || !aligned(heat, 4) || !aligned(scratch, 16))
     return SA_ERR_INVALID_ARG;
   const Geometry g = make_geometry(*desc);
   st = check_ws(g, workspace, ws_bytes);
   if (st != SA_OK) return st;
+  if (scratch_bytes < heat_scratch_bytes(g)) return SA_ERR_WORKSPACE;
   const WsLayout w = make_ws_layout(g);
   HeatArgs a;
   std::memset(&a, 0, sizeof(a));
@@ -179,6 +189,7 @@ sa_status sparse_attn_block_heatmap(const sa_desc* desc, const void* q, const vo
       !encode_tile_map(&a.map_k, k, g.BH, g.T, g.Hh, g.Ww, g.d, g.pt, g.ph, g.pw))
     return SA_ERR_CUDA;
   a.heat = heat;
+  a.scratch = static_cast<float*>(scratch);
   a.status = at<uint32_t>(workspace, w.status);
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)g.d));
   cudaStream_t s = static_cast<cudaStream_t>(stream);

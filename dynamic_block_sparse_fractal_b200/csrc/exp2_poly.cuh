@@ -67,4 +67,34 @@ __device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x) {
   return f2_pack(__uint_as_float(r_lo), __uint_as_float(r_hi));
 }
 
+// Degree-5 coefficients (gen_exp2_poly.py 5): max relative error 1.5e-7
+// after rounding them to fp32, on a par with ex2.approx; for sums that must
+// keep fp32-level accuracy.
+constexpr float kExp2D0 = 1.000000119e+00f;
+constexpr float kExp2D1 = 6.931469440e-01f;
+constexpr float kExp2D2 = 2.402212024e-01f;
+constexpr float kExp2D3 = 5.550713092e-02f;
+constexpr float kExp2D4 = 9.675540961e-03f;
+constexpr float kExp2D5 = 1.327647245e-03f;
+
+// 2^x for both lanes of x (each lane >= -125), degree-5 polynomial.
+__device__ __forceinline__ uint64_t exp2_poly5_x2(uint64_t x) {
+  const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);       // 1.5 * 2^23
+  const uint64_t neg_magic = f2_pack(-12582912.0f, -12582912.0f);
+  const uint64_t t = f2_add(x, magic);
+  const uint64_t n = f2_add(t, neg_magic);
+  const uint64_t f = f2_fma(n, f2_pack(-1.0f, -1.0f), x);
+  uint64_t p = f2_fma(f2_pack(kExp2D5, kExp2D5), f, f2_pack(kExp2D4, kExp2D4));
+  p = f2_fma(p, f, f2_pack(kExp2D3, kExp2D3));
+  p = f2_fma(p, f, f2_pack(kExp2D2, kExp2D2));
+  p = f2_fma(p, f, f2_pack(kExp2D1, kExp2D1));
+  p = f2_fma(p, f, f2_pack(kExp2D0, kExp2D0));
+  float p_lo, p_hi, t_lo, t_hi;
+  f2_unpack(p, p_lo, p_hi);
+  f2_unpack(t, t_lo, t_hi);
+  const uint32_t r_lo = __float_as_uint(p_lo) + (__float_as_uint(t_lo) << 23);
+  const uint32_t r_hi = __float_as_uint(p_hi) + (__float_as_uint(t_hi) << 23);
+  return f2_pack(__uint_as_float(r_lo), __uint_as_float(r_hi));
+}
+
 }  // namespace sa

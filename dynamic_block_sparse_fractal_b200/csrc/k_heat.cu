@@ -5,17 +5,26 @@
 // N x N block. A quality signal for a block mask: how much of the real
 // attention its kept blocks carry.
 //
-// One CTA per pair of consecutive q-blocks (a 128-row query tile), two dense
-// passes over all k-block pairs with S = Q K^T on the tensor cores:
-//   pass 1  the row's log-sum-exp: online max and sum of 2^x,
-//           x = s * log2(e) / sqrt(d), lse2 = m + log2(l);
-//   pass 2  per 64-key half (one k-block) the row max of x - lse2, reduced
-//           over the 64 rows of each q-block; H = 2^max.
-// warp 0: TMA (Q tile, then K pairs into a 3-slot ring, both passes);
-// warp 1: TMEM owner and MMA issuer (S double-buffered in TMEM);
-// warps 2-5: one thread per tile row (TMEM lane). All waits are bounded.
+// One dense pass over every key with S = Q K^T on the tensor cores. For a
+// query row r and a k-block b, H depends on the row only through
+//   max_{k in b} s[r][k]  and  lse2[r] = log2 sum_k 2^(x[r][k]),
+// x = s * log2(e) / sqrt(d):  H[qb][b] = max_{r in qb} 2^(xmax[r][b] - lse2[r]).
+// So each row keeps its online log-sum-exp (max m, sum l) and writes its raw
+// block maxima to a per-CTA fp32 scratch laid out [b][row]; once the row's
+// lse2 is final, its thread reads back its own entries, and the rows of a
+// q-block are reduced by a butterfly across the warp and an atomic max
+// (probabilities are non-negative, so their bits order like integers) on a
+// zeroed map.
+//
+// Persistent grid of at most kHeatCtas CTAs; a CTA's unit of work is four
+// consecutive q-blocks of one head as two 128-row query tiles A and B that
+// share every K pair. warp 0: TMA (Q tiles, K pairs into a 3-slot ring);
+// warp 1: TMEM owner (512 columns: S of A and B, double-buffered) and MMA
+// issuer; warps 2-5 / 6-9: one thread per row of tile A / B. All waits are
+// bounded.
 #include <cuda_runtime.h>
 
+#include "exp2_poly.cuh"
 #include "kernels.cuh"
 #include "sm100.cuh"
 
@@ -23,15 +32,22 @@ namespace sa {
 
 namespace {
 
-constexpr int kHThreads = 192;
+constexpr int kHThreads = 320;
 constexpr int kHSlots = 3;
-constexpr int kHChunk = 128 * 128;  // 128 rows x 128 B (64 bf16 channels)
+constexpr int kHChunk = 128 * 128;   // 128 rows x 128 B (64 bf16 channels)
+constexpr int kHRows = 256;          // scratch rows per CTA (two tiles)
+// Of every 8 column pairs of a row, this many take the FMA-pipe exp2 (degree
+// 5, fp32-level accuracy); the rest the special-function unit, which alone
+// would bound the pass.
+constexpr int kHeatPolyPairsPer8 = 3;
 
 template <int D>
 struct __align__(1024) HeatSmem {
-  uint8_t q[D / 64][kHChunk];
-  uint8_t slot[kHSlots][D / 64][kHChunk];
-  uint64_t q_full, full[kHSlots], empty[kHSlots], s_full[2], s_free[2], drain;
+  uint8_t q[2][D / 64][kHChunk];           // tiles A, B
+  uint8_t slot[kHSlots][D / 64][kHChunk];  // one K pair (128 keys) per slot
+  uint64_t q_full, q_empty, full[kHSlots], empty[kHSlots];
+  uint64_t s_full[2][2], s_free[2][2];  // [tile][TMEM buffer]
+  uint64_t drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -39,6 +55,14 @@ struct __align__(1024) HeatSmem {
 __device__ __forceinline__ void fail_h(uint32_t* status, int* abort, uint32_t bit) {
   atomicOr(status, bit);
   *reinterpret_cast<volatile int*>(abort) = 1;
+}
+
+// Unit u of the persistent loop: head bh, first q-block base (tile x, half h
+// holds q-block base + 2x + h, absent when >= nb).
+__device__ __forceinline__ void heat_unit(const Geometry& g, long u, int& bh, int& base) {
+  const int per_head = (g.nb + 3) / 4;
+  bh = int(u / per_head);
+  base = 4 * int(u - long(bh) * per_head);
 }
 
 }  // namespace
@@ -50,26 +74,26 @@ __global__ void __launch_bounds__(kHThreads, 1)
   HeatSmem<D>& sm = *reinterpret_cast<HeatSmem<D>*>(
       (reinterpret_cast<uintptr_t>(h_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.y;
-  const int qa = 2 * blockIdx.x, qb = qa + 1 < g.nb ? qa + 1 : -1;
-  const int nsteps = (g.nb + 1) / 2;  // k-block pairs per pass
-  const int nops = 2 * nsteps;
+  const long units = long(g.BH) * ((g.nb + 3) / 4);
+  const int nsteps = (g.nb + 1) / 2;  // K pairs per unit
   if (threadIdx.x == 0) {
     sm.abort = 0;
     mbar_init(&sm.q_full, 1);
+    mbar_init(&sm.q_empty, 1);
     for (int s = 0; s < kHSlots; ++s) {
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&sm.s_full[b], 1);
-      mbar_init(&sm.s_free[b], 128);
-    }
+    for (int x = 0; x < 2; ++x)
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&sm.s_full[x][b], 1);
+        mbar_init(&sm.s_free[x][b], 128);
+      }
     mbar_init(&sm.drain, 1);
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(&sm.tmem_base, 256);
+    tmem_alloc(&sm.tmem_base, 512);
     tmem_relinquish();
   }
   tc_fence_before_sync();
@@ -79,68 +103,96 @@ __global__ void __launch_bounds__(kHThreads, 1)
   volatile int* abort = &sm.abort;
 
   if (warp == 0) {
+    // ---------------------------------------------------------------- TMA
     if (lane == 0) {
       prefetch_tensormap(&a.map_q);
       prefetch_tensormap(&a.map_k);
-      mbar_arrive_expect_tx(&sm.q_full, 128u * D * 2u);
-      for (int e = 0; e < 2; ++e) {
-        const int blk = (e == 0 || qb < 0) ? qa : qb;
-        int t, hp, wp;
-        block_coords(g, blk, t, hp, wp);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_5d(&sm.q[c][e * 8192], &a.map_q, &sm.q_full, c * 64, wp * g.pw, hp * g.ph,
-                      t * g.pt, bh);
-      }
-      int issued = -1;
-      for (int m = 0; m < nops; ++m) {
-        const int s = m % kHSlots, use = m / kHSlots;
-        if (use > 0 && !mbar_wait(&sm.empty[s], (use - 1) & 1, abort)) {
+      int it = 0, op = 0, last_op = -1, last_q = -1;
+      for (long u = blockIdx.x; u < units && !*abort; u += gridDim.x, ++it) {
+        int bh, base;
+        heat_unit(g, u, bh, base);
+        if (it > 0 && !mbar_wait(&sm.q_empty, (it - 1) & 1, abort)) {
           fail_h(a.status, &sm.abort, kDevErrTimeoutLoad);
           break;
         }
-        if (*abort) break;
-        const int j = m % nsteps;
-        const int nblk = 2 * j + 1 < g.nb ? 2 : 1;
-        mbar_arrive_expect_tx(&sm.full[s], uint32_t(nblk) * 64u * D * 2u);
-        for (int e = 0; e < nblk; ++e) {
-          int t, hp, wp;
-          block_coords(g, 2 * j + e, t, hp, wp);
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_5d(&sm.slot[s][c][e * 8192], &a.map_k, &sm.full[s], c * 64, wp * g.pw,
-                        hp * g.ph, t * g.pt, bh);
+        mbar_arrive_expect_tx(&sm.q_full, 2u * 128u * D * 2u);
+        for (int x = 0; x < 2; ++x)
+          for (int e = 0; e < 2; ++e) {
+            const int blk = min(base + 2 * x + e, g.nb - 1);  // absent: any valid block
+            int t, hp, wp;
+            block_coords(g, blk, t, hp, wp);
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_5d(&sm.q[x][c][e * 8192], &a.map_q, &sm.q_full, c * 64, wp * g.pw,
+                          hp * g.ph, t * g.pt, bh);
+          }
+        last_q = it;
+        bool ok = true;
+        for (int j = 0; j < nsteps; ++j, ++op) {
+          const int s = op % kHSlots, use = op / kHSlots;
+          if (use > 0 && !mbar_wait(&sm.empty[s], (use - 1) & 1, abort)) {
+            fail_h(a.status, &sm.abort, kDevErrTimeoutLoad);
+            ok = false;
+            break;
+          }
+          if (*abort) {
+            ok = false;
+            break;
+          }
+          const int nblk = 2 * j + 1 < g.nb ? 2 : 1;
+          mbar_arrive_expect_tx(&sm.full[s], uint32_t(nblk) * 64u * D * 2u);
+          for (int e = 0; e < nblk; ++e) {
+            int t, hp, wp;
+            block_coords(g, 2 * j + e, t, hp, wp);
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_5d(&sm.slot[s][c][e * 8192], &a.map_k, &sm.full[s], c * 64, wp * g.pw,
+                          hp * g.ph, t * g.pt, bh);
+          }
+          last_op = op;
         }
-        issued = m;
+        if (!ok) break;
       }
-      if (*abort && issued >= 0) {  // let this thread's copies land before the CTA exits
+      if (*abort) {
+        // let this thread's copies land before the CTA can exit (time-bounded,
+        // ignoring the abort flag); at most one op per slot can be in flight
         int never = 0;
-        for (int m = issued; m >= 0 && m > issued - kHSlots; --m)
-          mbar_wait(&sm.full[m % kHSlots], (m / kHSlots) & 1, &never);
+        for (int o = last_op; o >= 0 && o > last_op - kHSlots; --o)
+          mbar_wait(&sm.full[o % kHSlots], (o / kHSlots) & 1, &never);
+        if (last_q >= 0) mbar_wait(&sm.q_full, last_q & 1, &never);
       }
     }
   } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA
     if (lane == 0) {
       const uint32_t id2 = idesc_bf16_f32(128, 128, 0, 0);
       const uint32_t id1 = idesc_bf16_f32(128, 64, 0, 0);
-      const uint64_t qd = sw128_desc(smem_u32(&sm.q[0][0]), 16, 1024);
+      const uint64_t qd0 = sw128_desc(smem_u32(&sm.q[0][0][0]), 16, 1024);
       const uint64_t kd0 = sw128_desc(smem_u32(&sm.slot[0][0][0]), 16, 1024);
-      constexpr uint32_t kSlotStep = (D / 64) * kHChunk / 16;
-      bool ok = mbar_wait(&sm.q_full, 0, abort);
-      for (int m = 0; ok && m < nops; ++m) {
-        const int s = m % kHSlots, buf = m & 1;
-        const int j = m % nsteps;
-        ok = mbar_wait(&sm.full[s], (m / kHSlots) & 1, abort) &&
-             (m < 2 || mbar_wait(&sm.s_free[buf], ((m >> 1) - 1) & 1, abort));
-        if (!ok) break;
-        tc_fence_after_sync();
-        const uint64_t kd = kd0 + uint64_t(s) * kSlotStep;
-        const uint32_t id = 2 * j + 1 < g.nb ? id2 : id1;
+      constexpr uint32_t kTileStep = (D / 64) * kHChunk / 16;  // descriptor units
+      bool ok = true;
+      int it = 0, op = 0;
+      for (long u = blockIdx.x; ok && u < units; u += gridDim.x, ++it) {
+        ok = mbar_wait(&sm.q_full, it & 1, abort);
+        for (int j = 0; ok && j < nsteps; ++j, ++op) {
+          const int s = op % kHSlots, buf = op & 1;
+          ok = mbar_wait(&sm.full[s], (op / kHSlots) & 1, abort);
+          const uint32_t id = 2 * j + 1 < g.nb ? id2 : id1;
+          const uint64_t kd = kd0 + uint64_t(s) * kTileStep;
+          for (int x = 0; ok && x < 2; ++x) {
+            ok = op < 2 || mbar_wait(&sm.s_free[x][buf], ((op >> 1) - 1) & 1, abort);
+            if (!ok) break;
+            tc_fence_after_sync();
+            const uint64_t qd = qd0 + uint64_t(x) * kTileStep;
+            const uint32_t d_tmem = tmem + uint32_t(x) * 256u + uint32_t(buf) * 128u;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (uint32_t(kk >> 2) * kHChunk + uint32_t(kk & 3) * 32u) >> 4;
-          mma_ss(tmem + uint32_t(buf) * 128u, qd + off, kd + off, id, kk > 0);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (uint32_t(kk >> 2) * kHChunk + uint32_t(kk & 3) * 32u) >> 4;
+              mma_ss(d_tmem, qd + off, kd + off, id, kk > 0);
+            }
+            mma_commit(&sm.s_full[x][buf]);
+          }
+          if (ok) mma_commit(&sm.empty[s]);
         }
-        mma_commit(&sm.empty[s]);
-        mma_commit(&sm.s_full[buf]);
+        if (ok) mma_commit(&sm.q_empty);
       }
       if (!ok) {
         fail_h(a.status, &sm.abort, kDevErrTimeoutMma);
@@ -150,67 +202,97 @@ __global__ void __launch_bounds__(kHThreads, 1)
       }
     }
   } else {
-    // processing: thread = tile row r (TMEM lane); rows 0-63 = qa, 64-127 = qb
-    const int quad = warp & 3;
+    // ---------------------------------------------------------------- rows
+    // thread = row r of tile x (TMEM lane r); rows 0-63 / 64-127 of a tile
+    // are its two q-blocks
+    const int x = (warp - 2) >> 2, quad = warp & 3;
     const int r = quad * 32 + lane;
     const int half = r >> 6;
-    const bool row_valid = half == 0 || qb >= 0;
-    const uint32_t t_lane = tmem + (uint32_t(quad * 32) << 16);
+    const uint32_t t_lane = tmem + (uint32_t(quad * 32) << 16) + uint32_t(x) * 256u;
+    // this thread's scratch column: entry b at mine[b * kHRows]
+    float* mine = a.scratch + size_t(blockIdx.x) * kHRows * g.nb + x * 128 + r;
     const float sl2 = a.scale_log2;
-    float m = -INFINITY, l = 0.f, lse2 = 0.f;
+    const uint64_t sl2x2 = f2_pack(sl2, sl2);
     bool ok = true;
-    for (int op = 0; op < nops; ++op) {
-      const int buf = op & 1, j = op % nsteps;
-      const int nblk = 2 * j + 1 < g.nb ? 2 : 1;
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sm.s_full[buf], (op >> 1) & 1, abort));
-      if (!ok) break;
-      tc_fence_after_sync();
-      uint32_t sv[128];
-      tmem_ld32(t_lane + buf * 128u + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-      tmem_ld32(t_lane + buf * 128u + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-      if (nblk == 2) {
-        tmem_ld32(t_lane + buf * 128u + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
-        tmem_ld32(t_lane + buf * 128u + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+    int op = 0;
+    for (long u = blockIdx.x; ok && u < units; u += gridDim.x) {
+      int bh, base;
+      heat_unit(g, u, bh, base);
+      float m = -INFINITY, l = 0.f;  // log2-domain running max and sum of the row
+      for (int j = 0; j < nsteps; ++j, ++op) {
+        const int buf = op & 1;
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sm.s_full[x][buf], (op >> 1) & 1, abort));
+        if (!ok) break;
+        tc_fence_after_sync();
+        const int nblk = 2 * j + 1 < g.nb ? 2 : 1;
+        for (int e = 0; e < nblk; ++e) {
+          uint32_t sv[64];
+          const uint32_t col = t_lane + uint32_t(buf) * 128u + uint32_t(e) * 64u;
+          tmem_ld32(col, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+          tmem_ld32(col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+          tmem_wait_ld();
+          if (e == nblk - 1) {
+            tc_fence_before_sync();
+            mbar_arrive(&sm.s_free[x][buf]);
+          }
+          // raw maximum of the row over k-block 2j + e (four chains)
+          float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int i = 0; i < 64; i += 2)
+            mq[(i >> 1) & 3] =
+                max3(mq[(i >> 1) & 3], __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
+          const float bmax = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+          mine[size_t(2 * j + e) * kHRows] = bmax;
+          const float m_new = fmaxf(m, bmax * sl2);
+          l *= ex2_approx(m - m_new);  // m = -inf at first: 2^-inf = 0
+          m = m_new;
+          // l += sum of 2^(s * sl2 - m) over the 64 columns, two per packed op
+          const uint64_t negm2 = f2_pack(-m, -m);
+          uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const uint64_t x2 =
+                f2_fma(f2_pack(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), sl2x2,
+                       negm2);
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            uint64_t e2;
+            if ((i & 7) >= 8 - kHeatPolyPairsPer8)
+              e2 = exp2_poly5_x2(f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f)));
+            else
+              e2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+            rs2[i & 3] = f2_add(rs2[i & 3], e2);
+          }
+          float lo, hi;
+          f2_unpack(f2_add(f2_add(rs2[0], rs2[1]), f2_add(rs2[2], rs2[3])), lo, hi);
+          l += lo + hi;
+        }
       }
-      tmem_wait_ld();
-      tc_fence_before_sync();
-      mbar_arrive(&sm.s_free[buf]);
-      if (op < nsteps) {
-        // pass 1: online log-sum-exp of x = s * log2(e) / sqrt(d)
-        float mx = -INFINITY;
+      if (!ok) break;
+      // ---- this unit's map rows: the row's lse2 is final
+      const float lse2 = m + __log2f(l);
+      const int qblk = base + 2 * x + half;  // uniform across the warp
+      if (qblk >= g.nb) continue;
+      int* out = reinterpret_cast<int*>(a.heat) + (size_t(bh) * g.nb + qblk) * g.nb;
+      for (int b0 = 0; b0 < g.nb; b0 += 32) {
+        float v[32];
 #pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (i < 64 * nblk) mx = fmaxf(mx, __uint_as_float(sv[i]) * sl2);
-        const float m_new = fmaxf(m, mx);
-        float sum = 0.f;
+        for (int i = 0; i < 32; ++i)
+          v[i] = b0 + i < g.nb ? fmaf(mine[size_t(b0 + i) * kHRows], sl2, -lse2) : -INFINITY;
+        // butterfly reduce-scatter over the warp's 32 rows: after the stage
+        // of width w, lane l holds in v[0..w) the maxima for the blocks whose
+        // index bits above w agree with l's; at the end v[0] = block b0 + lane
 #pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (i < 64 * nblk) sum += ex2_approx(__uint_as_float(sv[i]) * sl2 - m_new);
-        l = l * ex2_approx(m - m_new) + sum;  // m = -inf at first: 2^-inf = 0
-        m = m_new;
-        if (op == nsteps - 1) lse2 = m + __log2f(l);
-      } else {
-        // pass 2: per k-block, the max over this row of x - lse2, then over
-        // the warp's 32 rows; the two warps of a q-block meet in an atomic max
-        // on the (non-negative) probability's bits, on a zeroed map
-        float bm[2] = {-INFINITY, -INFINITY};
+        for (int w = 16; w >= 1; w >>= 1) {
+          const bool upper = (lane & w) != 0;
 #pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (i < 64 * nblk) bm[i >> 6] = fmaxf(bm[i >> 6], __uint_as_float(sv[i]) * sl2);
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          float v = bm[e] - lse2;
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-          bm[e] = v;
+          for (int i = 0; i < w; ++i) {
+            const float keep = upper ? v[i + w] : v[i];
+            const float send = upper ? v[i] : v[i + w];
+            v[i] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, send, w));
+          }
         }
-        if (lane < nblk && row_valid) {
-          const int qblk = half ? qb : qa;
-          const float p = ex2_approx(lane == 0 ? bm[0] : bm[1]);
-          atomicMax(reinterpret_cast<int*>(a.heat) + (size_t(bh) * g.nb + qblk) * g.nb + 2 * j +
-                        lane,
-                    __float_as_int(p));
-        }
+        if (b0 + lane < g.nb) atomicMax(out + b0 + lane, __float_as_int(ex2_approx(v[0])));
       }
     }
     if (!ok) fail_h(a.status, &sm.abort, kDevErrTimeoutSoftmax);
@@ -218,19 +300,19 @@ __global__ void __launch_bounds__(kHThreads, 1)
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
-  if (warp == 1) tmem_dealloc(tmem, 256);
+  if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
 template <int D>
 static cudaError_t launch_heat_d(const HeatArgs& a, const Geometry& g, cudaStream_t stream) {
-  const int smem = int(sizeof(HeatSmem<D>) + 1024);
+  // at least half the shared memory of an SM, so that one CTA (with its 512
+  // TMEM columns) is resident per SM whatever the register count
+  const int smem = max(int(sizeof(HeatSmem<D>) + 1024), 116 * 1024);
   cudaError_t e = cudaMemsetAsync(a.heat, 0, size_t(g.BH) * g.nb * g.nb * sizeof(float), stream);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(heat_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       smem);
+  e = cudaFuncSetAttribute(heat_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const dim3 grid(unsigned((g.nb + 1) / 2), unsigned(g.BH));
-  heat_kernel<D><<<grid, kHThreads, smem, stream>>>(a, g);
+  heat_kernel<D><<<unsigned(heat_ctas(g)), kHThreads, smem, stream>>>(a, g);
   return cudaGetLastError();
 }
 

@@ -60,13 +60,24 @@ struct AttnArgs {
 cudaError_t launch_attn(const AttnArgs& a, const Geometry& g, cudaStream_t stream);
 
 // Exact block max-pooled attention map: heat[bh][qb][kb] = max over the
-// block pair of the full softmax probability (zeroes heat, then one launch).
+// block pair of the full softmax probability (zeroes heat, then one launch of
+// a persistent grid of heat_ctas(g) CTAs, each with 256 rows of nb fp32 of
+// scratch).
 struct HeatArgs {
   CUtensorMap map_q, map_k;  // 5-D patch maps, one block per box
   float* heat;               // [BH][nb][nb], fractal block order
+  float* scratch;            // [heat_ctas(g)][nb][256]
   uint32_t* status;
   float scale_log2;  // log2(e) / sqrt(d)
 };
+constexpr int kHeatCtas = 148;  // one per SM of a B200
+inline int heat_ctas(const Geometry& g) {
+  const long units = long(g.BH) * ((g.nb + 3) / 4);  // four q-blocks each
+  return int(units < kHeatCtas ? units : kHeatCtas);
+}
+inline size_t heat_scratch_bytes(const Geometry& g) {
+  return size_t(heat_ctas(g)) * 256 * size_t(g.nb) * sizeof(float);
+}
 cudaError_t launch_heat(const HeatArgs& a, const Geometry& g, cudaStream_t stream);
 
 }  // namespace sa

@@ -235,17 +235,25 @@ sa_status sparse_attn_heads_run(const sa_desc* desc, const int* tiles, int run, 
  * head, max-pooled over every N x N block:
  *   heat[bh][i][j] = max over q in block i, k in block j of P[q][k],
  * blocks in fractal block order (the order of sparse_attn_get_mask's ids).
- * Computed exactly (dense, two passes over every key: the row log-sum-exp,
- * then the block maxima), so it costs about twice a dense QK^T; meant for
- * measuring a mask's recall, not for the attention path.
- * q, k: as for sparse_attn_plan. workspace: as for sparse_attn_plan; only its
+ * Computed exactly, densely (one pass over every key per query: about the
+ * cost of a dense Q K^T); meant for measuring a mask's recall, not for the
+ * attention path. */
+
+/* Bytes of device scratch sparse_attn_block_heatmap needs for `desc`
+ * (256 x nb fp32 per CTA of its grid, at most 148 CTAs). */
+sa_status sparse_attn_block_heatmap_scratch_size(const sa_desc* desc, size_t* bytes);
+
+/* q, k: as for sparse_attn_plan. workspace: as for sparse_attn_plan; only its
  * status word is used: cleared on `stream` before the launch, so the next
  * sparse_attn_check reports this call (a timed-out wait leaves heat
- * incomplete); the planned lists are left as they are. heat: device fp32 [B*H][nb][nb], 4-byte aligned,
- * owned by the caller, overwritten (zeroed first, on `stream`). */
+ * incomplete); the planned lists are left as they are. heat: device fp32
+ * [B*H][nb][nb], 4-byte aligned, owned by the caller, overwritten (zeroed
+ * first, on `stream`). scratch: device buffer of at least
+ * sparse_attn_block_heatmap_scratch_size() bytes, 16-byte aligned, contents
+ * ignored (SA_ERR_WORKSPACE when smaller). */
 sa_status sparse_attn_block_heatmap(const sa_desc* desc, const void* q, const void* k,
                                     void* workspace, size_t ws_bytes, float* heat,
-                                    void* stream);
+                                    void* scratch, size_t scratch_bytes, void* stream);
 
 #ifdef __cplusplus
 }

@@ -75,13 +75,19 @@ def test_entry_points_reject_before_launch():
     assert L.sparse_attn_check(ctypes.byref(d), FAKE, 0, None) == api.SA_ERR_WORKSPACE
     assert L.sparse_attn_get_mask(None, FAKE, need, ctypes.byref(v)) == api.SA_ERR_INVALID_ARG
     assert api.status_string(api.SA_ERR_DEVICE_TIMEOUT).startswith("a kernel")
-    st = L.sparse_attn_block_heatmap(ctypes.byref(d), FAKE, FAKE, FAKE, need, None, None)
-    assert st == api.SA_ERR_INVALID_ARG  # no heat buffer
-    st = L.sparse_attn_block_heatmap(ctypes.byref(d), FAKE, FAKE, FAKE, need,
-                                     ctypes.c_void_p(0x10000002), None)
-    assert st == api.SA_ERR_INVALID_ARG  # heat not 4-byte aligned
-    st = L.sparse_attn_block_heatmap(ctypes.byref(d), FAKE, FAKE, FAKE, need - 1, FAKE, None)
-    assert st == api.SA_ERR_WORKSPACE
+    sz = ctypes.c_size_t
+    scr = api.heatmap_scratch_size(d)
+    assert scr == 2 * 256 * 4 * 4  # two CTAs of 256 rows x 4 blocks (fp32)
+
+    def heat_call(ws_bytes, heat, scratch, scratch_bytes):
+        return L.sparse_attn_block_heatmap(ctypes.byref(d), FAKE, FAKE, FAKE, sz(ws_bytes), heat,
+                                           scratch, sz(scratch_bytes), None)
+    assert heat_call(need, None, FAKE, scr) == api.SA_ERR_INVALID_ARG  # no heat buffer
+    assert heat_call(need, ctypes.c_void_p(0x10000002), FAKE, scr) == \
+        api.SA_ERR_INVALID_ARG  # heat not 4-byte aligned
+    assert heat_call(need, FAKE, None, scr) == api.SA_ERR_INVALID_ARG  # no scratch
+    assert heat_call(need - 1, FAKE, FAKE, scr) == api.SA_ERR_WORKSPACE
+    assert heat_call(need, FAKE, FAKE, scr - 1) == api.SA_ERR_WORKSPACE
 
 
 @pytest.mark.parametrize("T,Hh,Ww", [(4, 8, 8), (33, 48, 80), (21, 32, 56), (3, 8, 24), (1, 16, 8)])
