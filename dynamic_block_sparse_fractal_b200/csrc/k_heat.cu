@@ -20,7 +20,8 @@
 // consecutive q-blocks of one head as two 128-row query tiles A and B that
 // share every K pair. warp 0: TMA (Q tiles, K pairs into a 3-slot ring);
 // warp 1: TMEM owner (512 columns: S of A and B, double-buffered) and MMA
-// issuer; warps 2-5 / 6-9: one thread per row of tile A / B. All waits are
+// issuer; warps 2-9 / 10-17: tile A / B, two threads per row, one per k-block
+// of each K pair (their running sums meet once per unit). All waits are
 // bounded.
 #include <cuda_runtime.h>
 
@@ -32,14 +33,14 @@ namespace sa {
 
 namespace {
 
-constexpr int kHThreads = 320;
+constexpr int kHThreads = 576;  // 2 control warps + 16 row warps
 constexpr int kHSlots = 3;
 constexpr int kHChunk = 128 * 128;   // 128 rows x 128 B (64 bf16 channels)
 constexpr int kHRows = 256;          // scratch rows per CTA (two tiles)
 // Of every 8 column pairs of a row, this many take the FMA-pipe exp2 (degree
 // 5, fp32-level accuracy); the rest the special-function unit, which alone
 // would bound the pass.
-constexpr int kHeatPolyPairsPer8 = 3;
+constexpr int kHeatPolyPairsPer8 = 2;
 
 template <int D>
 struct __align__(1024) HeatSmem {
@@ -47,10 +48,35 @@ struct __align__(1024) HeatSmem {
   uint8_t slot[kHSlots][D / 64][kHChunk];  // one K pair (128 keys) per slot
   uint64_t q_full, q_empty, full[kHSlots], empty[kHSlots];
   uint64_t s_full[2][2], s_free[2][2];  // [tile][TMEM buffer]
+  uint64_t lse_bar[2];                  // [tile]: both halves' (max, sum) written
   uint64_t drain;
+  float2 ml[2][2][2][128];              // [unit parity][tile][half][row]: (max, sum)
   uint32_t tmem_base;
   int abort;
 };
+
+// Sum over the 64 columns of 2^(s * sl2 - m), two columns per packed op;
+// kHeatPolyPairsPer8 of every 8 pairs take the FMA-pipe exp2.
+__device__ __forceinline__ float exp2_row_sum(const uint32_t (&sv)[64], uint64_t sl2x2, float m) {
+  const uint64_t negm2 = f2_pack(-m, -m);
+  uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const uint64_t x2 = f2_fma(
+        f2_pack(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), sl2x2, negm2);
+    float x0, x1;
+    f2_unpack(x2, x0, x1);
+    uint64_t e2;
+    if ((i & 7) >= 8 - kHeatPolyPairsPer8)
+      e2 = exp2_poly5_x2(f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f)));
+    else
+      e2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+    rs2[i & 3] = f2_add(rs2[i & 3], e2);
+  }
+  float lo, hi;
+  f2_unpack(f2_add(f2_add(rs2[0], rs2[1]), f2_add(rs2[2], rs2[3])), lo, hi);
+  return lo + hi;
+}
 
 __device__ __forceinline__ void fail_h(uint32_t* status, int* abort, uint32_t bit) {
   atomicOr(status, bit);
@@ -87,8 +113,9 @@ __global__ void __launch_bounds__(kHThreads, 1)
     for (int x = 0; x < 2; ++x)
       for (int b = 0; b < 2; ++b) {
         mbar_init(&sm.s_full[x][b], 1);
-        mbar_init(&sm.s_free[x][b], 128);
+        mbar_init(&sm.s_free[x][b], 256);
       }
+    for (int x = 0; x < 2; ++x) mbar_init(&sm.lse_bar[x], 256);
     mbar_init(&sm.drain, 1);
     fence_barrier_init();
   }
@@ -203,82 +230,77 @@ __global__ void __launch_bounds__(kHThreads, 1)
     }
   } else {
     // ---------------------------------------------------------------- rows
-    // thread = row r of tile x (TMEM lane r); rows 0-63 / 64-127 of a tile
+    // thread = row r of tile x (TMEM lane r), columns of k-block 2j + e of
+    // each step (e = which half of the K pair); rows 0-63 / 64-127 of a tile
     // are its two q-blocks
-    const int x = (warp - 2) >> 2, quad = warp & 3;
+    const int pw = warp - 2;
+    const int x = pw >> 3, e = (pw >> 2) & 1, quad = warp & 3;
     const int r = quad * 32 + lane;
     const int half = r >> 6;
-    const uint32_t t_lane = tmem + (uint32_t(quad * 32) << 16) + uint32_t(x) * 256u;
+    const uint32_t t_lane =
+        tmem + (uint32_t(quad * 32) << 16) + uint32_t(x) * 256u + uint32_t(e) * 64u;
     // this thread's scratch column: entry b at mine[b * kHRows]
     float* mine = a.scratch + size_t(blockIdx.x) * kHRows * g.nb + x * 128 + r;
     const float sl2 = a.scale_log2;
     const uint64_t sl2x2 = f2_pack(sl2, sl2);
     bool ok = true;
-    int op = 0;
-    for (long u = blockIdx.x; ok && u < units; u += gridDim.x) {
+    int op = 0, it = 0;
+    for (long u = blockIdx.x; ok && u < units; u += gridDim.x, ++it) {
       int bh, base;
       heat_unit(g, u, bh, base);
-      float m = -INFINITY, l = 0.f;  // log2-domain running max and sum of the row
+      float m = -INFINITY, l = 0.f;  // log2-domain running max and sum over this half
       for (int j = 0; j < nsteps; ++j, ++op) {
         const int buf = op & 1;
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sm.s_full[x][buf], (op >> 1) & 1, abort));
         if (!ok) break;
         tc_fence_after_sync();
-        const int nblk = 2 * j + 1 < g.nb ? 2 : 1;
-        for (int e = 0; e < nblk; ++e) {
-          uint32_t sv[64];
-          const uint32_t col = t_lane + uint32_t(buf) * 128u + uint32_t(e) * 64u;
-          tmem_ld32(col, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-          tmem_ld32(col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-          tmem_wait_ld();
-          if (e == nblk - 1) {
-            tc_fence_before_sync();
-            mbar_arrive(&sm.s_free[x][buf]);
-          }
-          // raw maximum of the row over k-block 2j + e (four chains)
-          float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-          for (int i = 0; i < 64; i += 2)
-            mq[(i >> 1) & 3] =
-                max3(mq[(i >> 1) & 3], __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
-          const float bmax = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
-          mine[size_t(2 * j + e) * kHRows] = bmax;
-          const float m_new = fmaxf(m, bmax * sl2);
-          l *= ex2_approx(m - m_new);  // m = -inf at first: 2^-inf = 0
-          m = m_new;
-          // l += sum of 2^(s * sl2 - m) over the 64 columns, two per packed op
-          const uint64_t negm2 = f2_pack(-m, -m);
-          uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const uint64_t x2 =
-                f2_fma(f2_pack(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), sl2x2,
-                       negm2);
-            float x0, x1;
-            f2_unpack(x2, x0, x1);
-            uint64_t e2;
-            if ((i & 7) >= 8 - kHeatPolyPairsPer8)
-              e2 = exp2_poly5_x2(f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f)));
-            else
-              e2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
-            rs2[i & 3] = f2_add(rs2[i & 3], e2);
-          }
-          float lo, hi;
-          f2_unpack(f2_add(f2_add(rs2[0], rs2[1]), f2_add(rs2[2], rs2[3])), lo, hi);
-          l += lo + hi;
+        if (2 * j + e >= g.nb) {  // the lone last k-block: nothing in this half
+          mbar_arrive(&sm.s_free[x][buf]);
+          continue;
         }
+        uint32_t sv[64];
+        tmem_ld32(t_lane + uint32_t(buf) * 128u, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(t_lane + uint32_t(buf) * 128u + 32u,
+                  *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_wait_ld();
+        tc_fence_before_sync();
+        mbar_arrive(&sm.s_free[x][buf]);
+        // raw maximum of the row over k-block 2j + e (four chains)
+        float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int i = 0; i < 64; i += 2)
+          mq[(i >> 1) & 3] =
+              max3(mq[(i >> 1) & 3], __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
+        const float bmax = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+        mine[size_t(2 * j + e) * kHRows] = bmax;
+        const float m_new = fmaxf(m, bmax * sl2);
+        l *= ex2_approx(m - m_new);  // m = -inf at first: 2^-inf = 0
+        m = m_new;
+        l += exp2_row_sum(sv, sl2x2, m);
       }
       if (!ok) break;
-      // ---- this unit's map rows: the row's lse2 is final
-      const float lse2 = m + __log2f(l);
+      // ---- the row's two halves meet: lse2 over all keys (both threads of
+      // the row compute the same value)
+      sm.ml[it & 1][x][e][r] = make_float2(m, l);
+      mbar_arrive(&sm.lse_bar[x]);
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sm.lse_bar[x], it & 1, abort));
+      if (!ok) break;
+      const float2 o = sm.ml[it & 1][x][e ^ 1][r];
+      const float mm = fmaxf(m, o.x);
+      const float ll = (e == 0 ? l * ex2_approx(m - mm) + o.y * ex2_approx(o.x - mm)
+                               : o.y * ex2_approx(o.x - mm) + l * ex2_approx(m - mm));
+      const float lse2 = mm + __log2f(ll);
+      // ---- this unit's map rows, blocks 2i + e
       const int qblk = base + 2 * x + half;  // uniform across the warp
       if (qblk >= g.nb) continue;
-      int* out = reinterpret_cast<int*>(a.heat) + (size_t(bh) * g.nb + qblk) * g.nb;
-      for (int b0 = 0; b0 < g.nb; b0 += 32) {
+      int* out = reinterpret_cast<int*>(a.heat) + (size_t(bh) * g.nb + qblk) * g.nb + e;
+      const int nbe = (g.nb - e + 1) / 2;  // blocks of this parity
+      for (int b0 = 0; b0 < nbe; b0 += 32) {
         float v[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i)
-          v[i] = b0 + i < g.nb ? fmaf(mine[size_t(b0 + i) * kHRows], sl2, -lse2) : -INFINITY;
+          v[i] = b0 + i < nbe ? fmaf(mine[size_t(2 * (b0 + i) + e) * kHRows], sl2, -lse2)
+                              : -INFINITY;
         // butterfly reduce-scatter over the warp's 32 rows: after the stage
         // of width w, lane l holds in v[0..w) the maxima for the blocks whose
         // index bits above w agree with l's; at the end v[0] = block b0 + lane
@@ -292,7 +314,7 @@ __global__ void __launch_bounds__(kHThreads, 1)
             v[i] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, send, w));
           }
         }
-        if (b0 + lane < g.nb) atomicMax(out + b0 + lane, __float_as_int(ex2_approx(v[0])));
+        if (b0 + lane < nbe) atomicMax(out + 2 * (b0 + lane), __float_as_int(ex2_approx(v[0])));
       }
     }
     if (!ok) fail_h(a.status, &sm.abort, kDevErrTimeoutSoftmax);
