@@ -244,6 +244,57 @@ def nabla_attention(q, k, v, T, Hh, Ww, P, N, thr, sta, mask=None):
     return out, mask
 
 
+# --- Gradients of the block-sparse attention (training use) -----------------
+# The NABLA page reuses the same block mask when training (pre-training and
+# fine-tuning a DiT, "Risultati Sperimentali"), which needs the gradients of
+# the masked attention: those of softmax attention with every dropped block at
+# -inf. With s = q.k / sqrt(d) on the kept blocks, P = softmax over a row's
+# kept keys and O = P V, for a loss with output gradient dO:
+#   dV = P^T dO,  dP = dO V^T,  D_i = sum_c dO_ic O_ic = sum_j P_ij dP_ij,
+#   dS = P * (dP - D),  dQ = dS K / sqrt(d),  dK = dS^T Q / sqrt(d).
+
+def masked_attention_backward(qp, kp, vp, dop, mask, N):
+    """Gradients of sum(O * dO) for O = masked_attention(qp, kp, vp, mask, N),
+    and the rows' natural-log log-sum-exp of the kept scaled scores.
+
+    qp, kp, vp, dop: [S, d] float64 (one head, fractal order); mask [nb, nb].
+    Returns (dq, dk, dv, lse): [S, d] x 3 and [S], fractal order.
+    """
+    S, d = qp.shape
+    scale = 1.0 / np.sqrt(d)
+    dq, dk, dv = np.zeros_like(qp), np.zeros_like(kp), np.zeros_like(vp)
+    lse = np.empty(S)
+    for qb in range(S // N):
+        r = slice(qb * N, (qb + 1) * N)
+        kept = np.nonzero(mask[qb])[0]
+        cols = (kept[:, None] * N + np.arange(N)[None, :]).reshape(-1)
+        s = qp[r] @ kp[cols].T * scale
+        mx = s.max(axis=-1, keepdims=True)
+        e = np.exp(s - mx)
+        l = e.sum(axis=-1, keepdims=True)
+        p = e / l
+        lse[r] = (mx + np.log(l))[:, 0]
+        o = p @ vp[cols]
+        dp = dop[r] @ vp[cols].T
+        D = (dop[r] * o).sum(axis=-1, keepdims=True)
+        ds = p * (dp - D)
+        dq[r] = ds @ kp[cols] * scale
+        dk[cols] += ds.T @ qp[r] * scale
+        dv[cols] += p.T @ dop[r]
+    return dq, dk, dv, lse
+
+
+def attention_backward_head(q, k, v, do, T, Hh, Ww, P, N, mask):
+    """One head in natural order: fractal flatten, masked_attention_backward,
+    inverse flatten. q, k, v, do: [S, d]. Returns (dq, dk, dv, lse) float64."""
+    perm = fractal_order(T, Hh, Ww, P)
+    qp, kp, vp, dop = (flatten(_as_f64(x), perm) for x in (q, k, v, do))
+    dq, dk, dv, lse = masked_attention_backward(qp, kp, vp, dop, mask, N)
+    lse_nat = np.empty_like(lse)
+    lse_nat[perm] = lse
+    return unflatten(dq, perm), unflatten(dk, perm), unflatten(dv, perm), lse_nat
+
+
 # --- Block max-pooled attention map (quality signal for a block mask) --------
 # The reference target of the page "Veda: Video Generation with Efficient
 # Sparse Attention", section 2.1 ("Costruzione dell'Obiettivo"): the full

@@ -442,9 +442,108 @@ def _mut_attention_no_scale(qp, kp, vp, mask, N, rows=None):
     return _orig_masked(qp * np.sqrt(qp.shape[-1]), kp, vp, mask, N, rows)
 
 
+def pin_backward_finite_differences(seed=41):
+    # Gradients of L = sum(O * G) against central differences of the forward
+    # oracle (itself pinned above), on a tiny head with a random block mask.
+    rng = np.random.default_rng(seed)
+    T, Hh, Ww, P, N, d = 2, 8, 16, 8, 64, 4
+    S = T * Hh * Ww
+    nb = S // N
+    q, k, v, g = (rng.standard_normal((S, d)) for _ in range(4))
+    mask = rng.random((nb, nb)) < 0.5
+    mask[np.arange(nb), np.arange(nb)] = True
+    perm = oracle.fractal_order(T, Hh, Ww, P)
+
+    def loss(q_, k_, v_):
+        qp, kp, vp = (oracle.flatten(x, perm) for x in (q_, k_, v_))
+        o = oracle.unflatten(oracle.masked_attention(qp, kp, vp, mask, N), perm)
+        return float((o * g).sum())
+
+    dq, dk, dv, _ = oracle.attention_backward_head(q, k, v, g, T, Hh, Ww, P, N, mask)
+    eps = 1e-6
+    for which, grad in ((0, dq), (1, dk), (2, dv)):
+        for _ in range(10):
+            i, c = int(rng.integers(S)), int(rng.integers(d))
+            args_p = [q.copy(), k.copy(), v.copy()]
+            args_m = [q.copy(), k.copy(), v.copy()]
+            args_p[which][i, c] += eps
+            args_m[which][i, c] -= eps
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+            assert abs(fd - grad[i, c]) < 1e-7 * max(1.0, abs(fd)), (which, i, c, fd, grad[i, c])
+
+
+def pin_backward_dense_is_torch_autograd(seed=43):
+    # With every block kept the gradients are those of plain softmax
+    # attention: torch's fp64 autograd of scaled_dot_product_attention.
+    import torch
+    rng = np.random.default_rng(seed)
+    T, Hh, Ww, P, N, d = 2, 8, 8, 8, 64, 8
+    S = T * Hh * Ww
+    q, k, v, g = (rng.standard_normal((S, d)) for _ in range(4))
+    mask = np.ones((S // N, S // N), dtype=bool)
+    dq, dk, dv, lse = oracle.attention_backward_head(q, k, v, g, T, Hh, Ww, P, N, mask)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    o = torch.nn.functional.scaled_dot_product_attention(tq[None], tk[None], tv[None])[0]
+    o.backward(torch.tensor(g))
+    for got, ref in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+        assert np.abs(got - ref.numpy()).max() < 1e-10
+    ref_lse = torch.logsumexp(torch.tensor(q) @ torch.tensor(k).T / np.sqrt(d), dim=-1)
+    assert np.abs(lse - ref_lse.numpy()).max() < 1e-10
+
+
+def pin_backward_uniform_rows():
+    # Zero queries: every kept score is 0, so lse = log(kept keys), P is
+    # uniform over the kept keys, dV of a key is the mean of dO over the rows
+    # that keep its block divided by their kept-key counts.
+    rng = np.random.default_rng(47)
+    T, Hh, Ww, P, N, d = 2, 8, 16, 8, 64, 4
+    S = T * Hh * Ww
+    nb = S // N
+    k, v, g = (rng.standard_normal((S, d)) for _ in range(3))
+    mask = rng.random((nb, nb)) < 0.5
+    mask[np.arange(nb), np.arange(nb)] = True
+    perm = oracle.fractal_order(T, Hh, Ww, P)
+    _, _, dv, lse = oracle.attention_backward_head(np.zeros((S, d)), k, v, g, T, Hh, Ww, P, N,
+                                                   mask)
+    kept_keys = mask.sum(axis=1) * N  # per q-block
+    lse_p = oracle.flatten(lse[:, None], perm)[:, 0]
+    assert np.allclose(lse_p, np.log(np.repeat(kept_keys, N)), rtol=0, atol=1e-12)
+    gp = oracle.flatten(g, perm)
+    expect = np.zeros((S, d))
+    for i in range(nb):
+        for j in np.nonzero(mask[i])[0]:
+            expect[j * N:(j + 1) * N] += gp[i * N:(i + 1) * N].sum(axis=0) / kept_keys[i]
+    assert np.abs(oracle.flatten(dv, perm) - expect).max() < 1e-12
+
+
 _orig_cdf = nabla.cdf_keep
 _orig_sta = nabla.sta_keep
 _orig_masked = nabla.masked_attention
+_orig_bwd = nabla.masked_attention_backward
+
+
+def _mut_backward_no_D(qp, kp, vp, dop, mask, N):
+    # dS = P * dP (the -D term dropped): only dQ and dK change
+    S, d = qp.shape
+    o = _orig_masked(qp, kp, vp, mask, N)
+    dq, dk, dv, lse = _orig_bwd(qp, kp, vp, dop, mask, N)
+    D = (dop * o).sum(axis=-1, keepdims=True)
+    # P * dP = dS + P * D: add the dropped term's contributions back
+    for qb in range(S // N):
+        r = slice(qb * N, (qb + 1) * N)
+        kept = np.nonzero(mask[qb])[0]
+        cols = (kept[:, None] * N + np.arange(N)[None, :]).reshape(-1)
+        s = qp[r] @ kp[cols].T / np.sqrt(d)
+        p = np.exp(s - s.max(axis=-1, keepdims=True))
+        p /= p.sum(axis=-1, keepdims=True)
+        dq[r] += (p * D[r]) @ kp[cols] / np.sqrt(d)
+        dk[cols] += (p * D[r]).T @ qp[r] / np.sqrt(d)
+    return dq, dk, dv, lse
+
+
+def _mut_backward_dk_unscaled(qp, kp, vp, dop, mask, N):
+    dq, dk, dv, lse = _orig_bwd(qp, kp, vp, dop, mask, N)
+    return dq, dk * np.sqrt(qp.shape[-1]), dv, lse
 
 MUTANTS = [
     ("fractal_order", _mut_fractal_inner_transposed, "fractal"),
@@ -459,7 +558,21 @@ MUTANTS = [
     ("sta_keep", _mut_sta_strict_distance, "sta"),
     ("masked_attention", _mut_attention_strided_blocks, "attention"),
     ("masked_attention", _mut_attention_no_scale, "attention"),
+    ("masked_attention_backward", _mut_backward_no_D, "backward"),
+    ("masked_attention_backward", _mut_backward_dk_unscaled, "backward"),
 ]
+
+
+def test_backward_finite_differences():
+    pin_backward_finite_differences()
+
+
+def test_backward_dense_is_torch_autograd():
+    pin_backward_dense_is_torch_autograd()
+
+
+def test_backward_uniform_rows():
+    pin_backward_uniform_rows()
 
 
 @pytest.mark.parametrize("name,mutant,area", MUTANTS, ids=[m[1].__name__ for m in MUTANTS])
@@ -474,6 +587,7 @@ def test_planted_mistake_is_caught(name, mutant, area, golden_dir, monkeypatch):
         "reduced": [pin_reduced_closed_form],
         "sta": [lambda: pin_sta_golden(golden_dir)],
         "attention": [pin_attention_own_patch, pin_attention_dense_is_sdpa],
+        "backward": [pin_backward_finite_differences, pin_backward_dense_is_torch_autograd],
     }[area]
     caught = 0
     for pin in pins:
