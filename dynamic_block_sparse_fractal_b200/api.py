@@ -29,7 +29,8 @@ SYMBOLS = (
     "sparse_attn_check", "sparse_attn_forward_noalloc", "sparse_attn_status_string",
     "sparse_attn_workspace_size_heads", "sparse_attn_plan_heads", "sparse_attn_fwd_heads",
     "sparse_attn_check_heads", "sparse_attn_heads_run", "sparse_attn_block_heatmap",
-    "sparse_attn_block_heatmap_scratch_size",
+    "sparse_attn_block_heatmap_scratch_size", "sparse_attn_fwd_lse",
+    "sparse_attn_bwd_scratch_size", "sparse_attn_bwd",
 )
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -188,6 +189,58 @@ def check(desc: SaDesc, workspace: torch.Tensor, stream=None) -> int:
     """Synchronises the stream; returns the status (SA_OK or an error code)."""
     return lib().sparse_attn_check(ctypes.byref(desc), _ptr(workspace), workspace.numel(),
                                    _stream(stream))
+
+
+def fwd_lse(desc: SaDesc, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+            workspace: torch.Tensor, out: torch.Tensor, lse: torch.Tensor,
+            stream=None) -> torch.Tensor:
+    """fwd that also writes each query row's log-sum-exp (fp32 [B, H, S])."""
+    _check_qkv(desc, q, k, v)
+    want = torch.float32 if desc.out_fp32 else torch.bfloat16
+    if out.dtype != want or out.shape != q.shape or not out.is_contiguous():
+        raise ValueError(f"out must be a contiguous {want} tensor shaped like q")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != tuple(q.shape[:3]) or \
+            not lse.is_contiguous():
+        raise ValueError(f"lse must be a contiguous float32 tensor of shape {tuple(q.shape[:3])}")
+    _ok(lib().sparse_attn_fwd_lse(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(workspace),
+                                  ctypes.c_size_t(workspace.numel()), _ptr(out), _ptr(lse),
+                                  _stream(stream)), "fwd_lse")
+    return out
+
+
+def bwd_scratch_size(desc: SaDesc) -> int:
+    n = ctypes.c_size_t(0)
+    _ok(lib().sparse_attn_bwd_scratch_size(ctypes.byref(desc), ctypes.byref(n)),
+        "bwd_scratch_size")
+    return n.value
+
+
+def bwd(desc: SaDesc, q, k, v, out, dout, lse, workspace, dq=None, dk=None, dv=None,
+        scratch=None, stream=None):
+    """Gradients (dq, dk, dv) of sum(out * dout) over the planned mask; see
+    include/sparse_attn.h. Allocates the outputs and the scratch when None."""
+    _check_qkv(desc, q, k, v, dout)
+    want = torch.float32 if desc.out_fp32 else torch.bfloat16
+    if out.dtype != want or out.shape != q.shape or not out.is_contiguous():
+        raise ValueError(f"out must be a contiguous {want} tensor shaped like q")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != tuple(q.shape[:3]) or \
+            not lse.is_contiguous():
+        raise ValueError(f"lse must be a contiguous float32 tensor of shape {tuple(q.shape[:3])}")
+    grads = []
+    for g in (dq, dk, dv):
+        if g is None:
+            g = torch.empty(q.shape, dtype=want, device=q.device)
+        if g.dtype != want or g.shape != q.shape or not g.is_contiguous():
+            raise ValueError(f"gradients must be contiguous {want} tensors shaped like q")
+        grads.append(g)
+    if scratch is None:
+        scratch = torch.empty(bwd_scratch_size(desc), dtype=torch.uint8, device=q.device)
+    _ok(lib().sparse_attn_bwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                              _ptr(dout), _ptr(lse), _ptr(workspace),
+                              ctypes.c_size_t(workspace.numel()), _ptr(grads[0]), _ptr(grads[1]),
+                              _ptr(grads[2]), _ptr(scratch), ctypes.c_size_t(scratch.numel()),
+                              _stream(stream)), "bwd")
+    return tuple(grads)
 
 
 def heatmap_scratch_size(desc: SaDesc) -> int:

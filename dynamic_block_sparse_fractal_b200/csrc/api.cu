@@ -131,8 +131,9 @@ sa_status sparse_attn_plan(const sa_desc* desc, const void* q, const void* k, vo
   return cuda_status(launch_tile_order(m.tcnt, at<int32_t>(workspace, w.order), g, s));
 }
 
-sa_status sparse_attn_fwd(const sa_desc* desc, const void* q, const void* k, const void* v,
-                          const void* workspace, size_t ws_bytes, void* out, void* stream) {
+static sa_status fwd_impl(const sa_desc* desc, const void* q, const void* k, const void* v,
+                          const void* workspace, size_t ws_bytes, void* out, float* lse,
+                          void* stream) {
   sa_status st = validate(desc);
   if (st != SA_OK) return st;
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || !aligned(q, 16) ||
@@ -159,7 +160,76 @@ sa_status sparse_attn_fwd(const sa_desc* desc, const void* q, const void* k, con
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)g.d));
   a.out_fp32 = desc->out_fp32;
   a.debug_flags = desc->debug_flags;
+  a.lse = lse;
   return cuda_status(launch_attn(a, g, static_cast<cudaStream_t>(stream)));
+}
+
+sa_status sparse_attn_fwd(const sa_desc* desc, const void* q, const void* k, const void* v,
+                          const void* workspace, size_t ws_bytes, void* out, void* stream) {
+  return fwd_impl(desc, q, k, v, workspace, ws_bytes, out, nullptr, stream);
+}
+
+sa_status sparse_attn_fwd_lse(const sa_desc* desc, const void* q, const void* k, const void* v,
+                              const void* workspace, size_t ws_bytes, void* out, float* lse,
+                              void* stream) {
+  if (lse == nullptr || !aligned(lse, 4)) return SA_ERR_INVALID_ARG;
+  return fwd_impl(desc, q, k, v, workspace, ws_bytes, out, lse, stream);
+}
+
+sa_status sparse_attn_bwd_scratch_size(const sa_desc* desc, size_t* bytes) {
+  const sa_status st = validate(desc);
+  if (st != SA_OK) return st;
+  if (bytes == nullptr) return SA_ERR_INVALID_ARG;
+  *bytes = make_bwd_layout(make_geometry(*desc)).total;
+  return SA_OK;
+}
+
+sa_status sparse_attn_bwd(const sa_desc* desc, const void* q, const void* k, const void* v,
+                          const void* out, const void* dout, const float* lse,
+                          const void* workspace, size_t ws_bytes, void* dq, void* dk, void* dv,
+                          void* scratch, size_t scratch_bytes, void* stream) {
+  sa_status st = validate(desc);
+  if (st != SA_OK) return st;
+  const void* ptrs[] = {q, k, v, out, dout, dq, dk, dv, scratch};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned(p, 16)) return SA_ERR_INVALID_ARG;
+  if (lse == nullptr || !aligned(lse, 4)) return SA_ERR_INVALID_ARG;
+  const Geometry g = make_geometry(*desc);
+  st = check_ws(g, workspace, ws_bytes);
+  if (st != SA_OK) return st;
+  const BwdLayout b = make_bwd_layout(g);
+  if (scratch_bytes < b.total) return SA_ERR_WORKSPACE;
+  if (!aligned(scratch, 256)) return SA_ERR_INVALID_ARG;
+  const WsLayout w = make_ws_layout(g);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  BwdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  if (!encode_tile_map(&a.map_q, q, g.BH, g.T, g.Hh, g.Ww, g.d, g.pt, g.ph, g.pw) ||
+      !encode_tile_map(&a.map_k, k, g.BH, g.T, g.Hh, g.Ww, g.d, g.pt, g.ph, g.pw) ||
+      !encode_tile_map(&a.map_v, v, g.BH, g.T, g.Hh, g.Ww, g.d, g.pt, g.ph, g.pw) ||
+      !encode_tile_map(&a.map_do, dout, g.BH, g.T, g.Hh, g.Ww, g.d, g.pt, g.ph, g.pw))
+    return SA_ERR_CUDA;
+  a.lse2 = at<float>(scratch, b.lse2);
+  a.dsum = at<float>(scratch, b.dsum);
+  a.kcnt = at<int32_t>(scratch, b.kcnt);
+  a.kidx = at<int32_t>(scratch, b.kidx);
+  a.dq_acc = at<float>(scratch, b.dq_acc);
+  a.dk = dk;
+  a.dv = dv;
+  a.status = const_cast<uint32_t*>(at<uint32_t>(workspace, w.status));
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)g.d));
+  a.scale = (float)(1.0 / std::sqrt((double)g.d));
+  a.out_fp32 = desc->out_fp32;
+  cudaError_t e = cudaMemsetAsync(a.dq_acc, 0, sizeof(float) * size_t(g.BH) * g.S * g.d, s);
+  if (e == cudaSuccess)
+    e = launch_bwd_prep(out, dout, lse, at<float>(scratch, b.lse2), at<float>(scratch, b.dsum),
+                        desc->out_fp32, g, s);
+  if (e == cudaSuccess)
+    e = launch_bwd_lists(at<uint32_t>(workspace, w.bits), at<int32_t>(scratch, b.kcnt),
+                         at<int32_t>(scratch, b.kidx), g, s);
+  if (e == cudaSuccess) e = launch_bwd(a, g, s);
+  if (e == cudaSuccess) e = launch_dq_convert(a.dq_acc, dq, desc->out_fp32, g, s);
+  return cuda_status(e);
 }
 
 sa_status sparse_attn_block_heatmap_scratch_size(const sa_desc* desc, size_t* bytes) {

@@ -518,6 +518,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                              size_t(wp * g.pw + (i & (g.pw - 1)));
           const size_t row = size_t(bh) * g.S + tok;
           const float inv = l > 0.f ? 1.0f / l : 0.f;
+          // log-sum-exp of the row's kept scaled scores (natural log): m is
+          // in log2 units and l is the sum relative to 2^m
+          if (a.lse != nullptr)
+            a.lse[row] = l > 0.f ? (m + __log2f(l)) * 0.6931471805599453f : -INFINITY;
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];

@@ -56,6 +56,7 @@ struct AttnArgs {
   float scale_log2;  // log2(e) / sqrt(d)
   int out_fp32;
   int debug_flags;
+  float* lse;  // [BH][S] natural order: each row's log-sum-exp (natural log), or null
 };
 cudaError_t launch_attn(const AttnArgs& a, const Geometry& g, cudaStream_t stream);
 
@@ -70,6 +71,54 @@ struct HeatArgs {
   uint32_t* status;
   float scale_log2;  // log2(e) / sqrt(d)
 };
+// Gradients of the block-sparse attention. Scratch (every region 256-byte
+// aligned): dq_acc fp32 [BH][S][d] natural order (zeroed, then reduced into),
+// lse2 and dsum fp32 [BH][S] in fractal order, kcnt int32 [BH][ntile] and
+// kidx int32 [BH][ntile][nb]: per key tile (the query-tile pairing applied to
+// k-blocks) the q-blocks keeping either of its k-blocks, ascending, as
+// q-block | kEntryKeepA (keeps the first k-block) | kEntryKeepB (the second).
+struct BwdLayout {
+  size_t dq_acc, lse2, dsum, kcnt, kidx, total;
+};
+inline BwdLayout make_bwd_layout(const Geometry& g) {
+  BwdLayout b;
+  size_t o = 0;
+  b.dq_acc = o; o = align256(o + sizeof(float) * size_t(g.BH) * g.S * g.d);
+  b.lse2 = o; o = align256(o + sizeof(float) * size_t(g.BH) * g.S);
+  b.dsum = o; o = align256(o + sizeof(float) * size_t(g.BH) * g.S);
+  b.kcnt = o; o = align256(o + sizeof(int32_t) * size_t(g.BH) * g.ntile);
+  b.kidx = o; o = align256(o + sizeof(int32_t) * size_t(g.BH) * g.ntile * g.nb);
+  b.total = o;
+  return b;
+}
+
+struct BwdArgs {
+  CUtensorMap map_q, map_k, map_v, map_do;  // 5-D patch maps, one block per box
+  const float* lse2;                        // [BH][S] fractal order, log2 units
+  const float* dsum;                        // [BH][S] fractal order: rowsum(dO * O)
+  const int32_t* kcnt;
+  const int32_t* kidx;
+  float* dq_acc;  // [BH][S][d] natural order, zeroed
+  void* dk;       // [BH][S][d] natural order, bf16 or fp32
+  void* dv;
+  uint32_t* status;
+  float scale_log2;  // log2(e) / sqrt(d)
+  float scale;       // 1 / sqrt(d)
+  int out_fp32;
+};
+// D = rowsum(dO * O) and lse * log2(e), both into fractal order (o: bf16 or
+// fp32 per o_fp32; do_: bf16; lse: natural-log row log-sum-exp, natural order).
+cudaError_t launch_bwd_prep(const void* o, const void* do_, const float* lse, float* lse2,
+                            float* dsum, int o_fp32, const Geometry& g, cudaStream_t stream);
+// Per key tile, the q-blocks that keep one of its k-blocks (from the keep bitmaps).
+cudaError_t launch_bwd_lists(const uint32_t* bits, int32_t* kcnt, int32_t* kidx, const Geometry& g,
+                             cudaStream_t stream);
+// dK, dV of every key tile and dQ reduced into dq_acc.
+cudaError_t launch_bwd(const BwdArgs& a, const Geometry& g, cudaStream_t stream);
+// dq = dq_acc (bf16 or fp32).
+cudaError_t launch_dq_convert(const float* dq_acc, void* dq, int out_fp32, const Geometry& g,
+                              cudaStream_t stream);
+
 constexpr int kHeatCtas = 148;  // one per SM of a B200
 inline int heat_ctas(const Geometry& g) {
   const long units = long(g.BH) * ((g.nb + 3) / 4);  // four q-blocks each

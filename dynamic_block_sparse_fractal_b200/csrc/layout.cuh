@@ -57,6 +57,17 @@ SA_HD void block_coords(const Geometry& g, int b, int& t, int& hp, int& wp) {
   wp = r - hp * g.nw;
 }
 
+// Natural token index (within a head) of row i (0..63) of block b: frame
+// t*pt + (i >> (lph + lpw)), row hp*ph + ((i >> lpw) & (ph - 1)), column
+// wp*pw + (i & (pw - 1)).
+SA_HD int block_row_token(const Geometry& g, int b, int i) {
+  int t, hp, wp;
+  block_coords(g, b, t, hp, wp);
+  const int run = i >> g.lpw;
+  return (t * g.pt + (run >> g.lph)) * g.Hh * g.Ww + (hp * g.ph + (run & (g.ph - 1))) * g.Ww +
+         wp * g.pw + (i & (g.pw - 1));
+}
+
 // Query tile -> the two q-blocks it holds (qb = -1 when alone). Pairs are
 // the same patch in block frames (2i, 2i+1); an odd last block frame pairs
 // neighbouring patch columns.

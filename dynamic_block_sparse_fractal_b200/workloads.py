@@ -187,3 +187,17 @@ def make_inputs(w: Workload, heads: Optional[range] = None):
     if heads is None:
         return tuple(o.reshape(w.B, w.H, w.S, w.d) for o in out)
     return tuple(out)
+
+
+def make_output_grad(w: Workload, heads: Optional[range] = None) -> np.ndarray:
+    """A seeded upstream gradient dO for the workload's output: i.i.d. standard
+    normal values as bf16 bits, [B, H, S, d] (or [len(heads), S, d]); a head's
+    values do not depend on which other heads are generated."""
+    rng = np.random.Generator(np.random.PCG64(w.seed ^ 0x5EED_0D0))
+    head_seeds = rng.integers(0, 2**63 - 1, size=w.BH)
+    sel = range(w.BH) if heads is None else heads
+    out = np.empty((len(sel), w.S, w.d), dtype=np.uint16)
+    for i, bh in enumerate(sel):
+        hr = np.random.Generator(np.random.PCG64(int(head_seeds[bh])))
+        out[i] = f32_to_bf16_bits(hr.standard_normal((w.S, w.d), dtype=np.float32))
+    return out.reshape(w.B, w.H, w.S, w.d) if heads is None else out

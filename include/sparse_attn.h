@@ -228,6 +228,39 @@ sa_status sparse_attn_check_heads(const sa_desc* desc, const int* tiles, const v
 sa_status sparse_attn_heads_run(const sa_desc* desc, const int* tiles, int run, sa_desc* sub,
                                 int* head0, size_t* ws_offset, size_t* ws_bytes);
 
+/* ---- Gradients (training use of the mask) ---------------------------------
+ * The NABLA page uses the same block mask when training a DiT ("Risultati
+ * Sperimentali"), which needs the gradients of the masked attention. With
+ * s = q.k / sqrt(d) on the kept blocks, P the softmax over a row's kept keys
+ * and O = P V:  dV = P^T dO, dP = dO V^T, D_i = sum_c dO_ic O_ic,
+ * dS = P (dP - D), dQ = dS K / sqrt(d), dK = dS^T Q / sqrt(d). */
+
+/* sparse_attn_fwd that also writes each query row's log-sum-exp of its kept
+ * scaled scores (natural log) to lse: device fp32 [B*H][S], natural token
+ * order, 4-byte aligned. */
+sa_status sparse_attn_fwd_lse(const sa_desc* desc, const void* q, const void* k,
+                              const void* v, const void* workspace, size_t ws_bytes,
+                              void* out, float* lse, void* stream);
+
+/* Bytes of device scratch sparse_attn_bwd needs: an fp32 dQ accumulator
+ * [B*H][S][d], two fp32 [B*H][S] row statistics and the transposed block
+ * lists (int32 [B*H][ntile] counts and [B*H][ntile][nb] entries). */
+sa_status sparse_attn_bwd_scratch_size(const sa_desc* desc, size_t* bytes);
+
+/* dq, dk, dv = gradients of sum(out * dout) with respect to q, k, v, over the
+ * mask of the plan in `workspace` (made for the same desc; its status word
+ * collects device timeouts, see sparse_attn_check). q, k, v: as for
+ * sparse_attn_fwd; out, lse: what sparse_attn_fwd_lse wrote for them (out
+ * bf16, or fp32 if desc->out_fp32); dout: [B,H,S,d] bf16 (it is a
+ * tensor-core operand). dq, dk, dv: [B,H,S,d], natural order, bf16 (fp32 if
+ * desc->out_fp32), overwritten. scratch: at least
+ * sparse_attn_bwd_scratch_size() bytes, 256-byte aligned, contents ignored.
+ * All tensor pointers 16-byte aligned (lse 4). */
+sa_status sparse_attn_bwd(const sa_desc* desc, const void* q, const void* k, const void* v,
+                          const void* out, const void* dout, const float* lse,
+                          const void* workspace, size_t ws_bytes, void* dq, void* dk,
+                          void* dv, void* scratch, size_t scratch_bytes, void* stream);
+
 /* ---- Block max-pooled attention map (mask diagnostics) -------------------
  * "Veda: Video Generation with Efficient Sparse Attention", section 2.1
  * ("Costruzione dell'Obiettivo"): the reference a block mask is judged

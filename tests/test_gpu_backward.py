@@ -1,0 +1,85 @@
+"""Gradients of the block-sparse attention (through the C ABI) against the
+fp64 oracle, on the GPU's own mask, and the row log-sum-exp of the forward.
+
+Tolerances. The kernel recomputes P = 2^(s log2(e) - lse2) in fp32, rounds P
+and dS = P (dP - D) to bf16 for the tensor cores (relative 2^-9 each) and
+accumulates in fp32; D = rowsum(dO * O) uses the forward's output as stored
+(bf16 unless out_fp32), which moves D by up to 2^-9 of |O|. Errors are
+measured relative to the largest reference magnitude of each gradient:
+max |g - ref| <= REL_MAX * max |ref| and mean |g - ref| <= REL_MEAN * mean |ref|.
+dQ and dK are the loosest: a row's dS sums to about zero (sum_j P (dP - D) = 0),
+so the bf16 rounding of its terms is large next to the sums they form. Seen on
+these cases: max 1.2e-2 (dQ), mean 6.0e-3 with bf16 outputs (their own
+rounding adds ~2^-10 on average) and 2.9e-3 with fp32 outputs; the bounds
+leave about a factor two.
+"""
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from dynamic_block_sparse_fractal_b200 import api, workloads as W
+from tests import parity
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+REL_MAX = {False: 2.5e-2, True: 2.5e-2}    # keyed by out_fp32
+REL_MEAN = {False: 1.2e-2, True: 6e-3}
+LSE_ABS = 1e-4
+
+CASES = [
+    W.TINY,
+    W.TINY.with_(name="odd_1x2x576x128", T=3, Hh=8, Ww=24, d=128),
+    W.W8K_T248.with_(name="tile2x4x8_1x2x4096x128", T=8, Hh=16, Ww=32, H=2),
+    W.W8K.with_(name="8k_1x2x8192x128_sta3", H=2),
+]
+
+
+def to_dev(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+@functools.lru_cache(maxsize=4)
+def gpu_grads(w, out_fp32):
+    q, k, v = W.make_inputs(w)
+    g = W.make_output_grad(w)
+    qd, kd, vd, gd = (to_dev(x) for x in (q, k, v, g))
+    desc = api.desc_for(w, out_fp32=out_fp32)
+    ws = api.alloc_workspace(desc)
+    api.plan(desc, qd, kd, ws)
+    out = torch.empty(qd.shape, device="cuda",
+                      dtype=torch.float32 if out_fp32 else torch.bfloat16)
+    lse = torch.empty(qd.shape[:3], dtype=torch.float32, device="cuda")
+    api.fwd_lse(desc, qd, kd, vd, ws, out, lse)
+    dq, dk, dv = api.bwd(desc, qd, kd, vd, out, gd, lse, ws)
+    st = api.check(desc, ws)
+    assert st == api.SA_OK, api.status_string(st)
+    views = api.get_mask(desc, ws)
+    mask = parity.lists_to_mask(views["cnt"].cpu().numpy(), views["idx"].cpu().numpy())
+    host = lambda t: t.float().cpu().numpy().reshape(w.BH, w.S, w.d)
+    return (host(dq), host(dk), host(dv), lse.cpu().numpy().reshape(w.BH, w.S), mask)
+
+
+def rel_errors(got, ref):
+    e = np.abs(got - ref)
+    return e.max() / np.abs(ref).max(), e.mean() / np.abs(ref).mean()
+
+
+@pytest.mark.parametrize("out_fp32", [False, True])
+@pytest.mark.parametrize("w", CASES, ids=[c.name for c in CASES])
+def test_backward_matches_oracle(w, out_fp32):
+    dq, dk, dv, lse, mask = gpu_grads(w, out_fp32)
+    q, k, v = (x.reshape(w.BH, w.S, w.d) for x in W.make_inputs(w))
+    g = W.make_output_grad(w).reshape(w.BH, w.S, w.d)
+    for bh in range(w.BH):
+        rq, rk, rv, rl = oracle.attention_backward_head(q[bh], k[bh], v[bh], g[bh], w.T, w.Hh,
+                                                        w.Ww, w.block, w.N, mask[bh])
+        assert np.abs(lse[bh] - rl).max() < LSE_ABS
+        for name, got, ref in (("dq", dq[bh], rq), ("dk", dk[bh], rk), ("dv", dv[bh], rv)):
+            mx, mean = rel_errors(got, ref)
+            print(f"{w.name} fp32={out_fp32} head {bh} {name}: max {mx:.2e} mean {mean:.2e}")
+            assert mx <= REL_MAX[out_fp32], (name, bh, mx)
+            assert mean <= REL_MEAN[out_fp32], (name, bh, mean)
