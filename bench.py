@@ -282,6 +282,8 @@ def run_ours(args, w, rank, world):
 
     heatmap = None if args.no_heatmap else measure_heatmap(api, desc, w, q, k, ws, views, dev,
                                                              stream)
+    backward = None if args.no_backward else measure_backward(api, desc, w, q, k, v, ws,
+                                                              kept_pairs, dev, stream)
 
     peaks, src = load_peaks()
     ms_step = total_ms / args.steps
@@ -317,6 +319,9 @@ def run_ours(args, w, rank, world):
     if heatmap is not None:
         heatmap["frac"] = round(heatmap["tensor_tflops"] / peak, 4)
         line["heatmap"] = heatmap
+    if backward is not None:
+        backward["frac"] = round(backward["kept_tflops"] / peak, 4)
+        line["backward"] = backward
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -353,6 +358,36 @@ def measure_heatmap(api, desc, w, q, k, ws, views, dev, stream, reps=3):
             "note": "one dense Q K^T pass (row log-sum-exp + raw block maxima, then per-row "
                     "reduction of the maxima); time includes zeroing the map",
             "mask_recall": round(recall, 4)}
+
+
+def measure_backward(api, desc, w, q, k, v, ws, kept_pairs, dev, stream, reps=3):
+    """Times sparse_attn_bwd (prep, transposed lists, the gradient kernel, dQ
+    conversion) on the planned mask with a seeded upstream gradient, outside
+    the step. Kept FLOPs: five N x N x d GEMMs per kept (q-block, k-block) pair
+    (S, dP, dV, dK, dQ)."""
+    import torch
+    g = to_device(W.make_output_grad(w), w, dev)
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    api.fwd_lse(desc, q, k, v, ws, out, lse)
+    grads = [torch.empty_like(q) for _ in range(3)]
+    scratch = torch.empty(api.bwd_scratch_size(desc), dtype=torch.uint8, device=dev)
+    api.bwd(desc, q, k, v, out, g, lse, ws, *grads, scratch=scratch)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(reps):
+        api.bwd(desc, q, k, v, out, g, lse, ws, *grads, scratch=scratch)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / reps
+    st = api.check(desc, ws)
+    if st != api.SA_OK:
+        raise SystemExit(f"device status after the backward: {api.status_string(st)}")
+    flops = kept_pairs * 5 * kept_flops_per_pair(w) / 2  # kept_flops_per_pair counts 2 GEMMs
+    return {"kernels": "bwd_prep, bwd_lists, sa::bwd_kernel<%d>, dq_convert" % w.d,
+            "ms": round(ms, 3), "kept_tflops": round(flops / (ms * 1e-3) / 1e12, 2),
+            "note": "one sparse_attn_bwd call: dQ, dK, dV over the planned mask"}
 
 
 def oracle_sample(w, budget_s=20.0, seed=0):
@@ -425,6 +460,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-heatmap", action="store_true",
                     help="skip the block max-pooled attention map measurement")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the gradient (backward) measurement")
     ap.add_argument("--heads", type=int, default=None,
                     help="run the workload's grid with this many heads (small ncu captures); "
                          "the line's config then names the changed workload")

@@ -8,5 +8,5 @@ from .nabla import (  # noqa: F401
     widen_bf16, fractal_order, flatten, unflatten, pool, reduced_map, cdf_keep,
     block_coords, sta_keep, pooled_head, nabla_mask, masked_attention,
     attention_head, nabla_attention, tile_shape, block_heatmap, block_heatmap_rows, heat_recall,
-    masked_attention_backward, attention_backward_head,
+    masked_attention_backward, masked_attention_backward_blocks, attention_backward_head,
 )

@@ -284,6 +284,45 @@ def masked_attention_backward(qp, kp, vp, dop, mask, N):
     return dq, dk, dv, lse
 
 
+def masked_attention_backward_blocks(qp, kp, vp, dop, mask, N, qblocks, kblocks):
+    """The rows of masked_attention_backward for some blocks only: dq of the
+    q-blocks ``qblocks`` and dk, dv of the k-blocks ``kblocks``, from the
+    q-blocks involved (those sampled, and those keeping a sampled k-block).
+    Returns (dq [len(qblocks), N, d], dk, dv [len(kblocks), N, d], lse
+    [len(qblocks), N]), fractal order within each block."""
+    S, d = qp.shape
+    scale = 1.0 / np.sqrt(d)
+    qblocks, kblocks = list(qblocks), list(kblocks)
+    dq = np.zeros((len(qblocks), N, d))
+    lse = np.zeros((len(qblocks), N))
+    dk = np.zeros((len(kblocks), N, d))
+    dv = np.zeros((len(kblocks), N, d))
+    rows = set(qblocks) | {int(i) for b in kblocks for i in np.nonzero(mask[:, b])[0]}
+    for qb in sorted(rows):
+        r = slice(qb * N, (qb + 1) * N)
+        kept = np.nonzero(mask[qb])[0]
+        cols = (kept[:, None] * N + np.arange(N)[None, :]).reshape(-1)
+        s = qp[r] @ kp[cols].T * scale
+        mx = s.max(axis=-1, keepdims=True)
+        e = np.exp(s - mx)
+        l = e.sum(axis=-1, keepdims=True)
+        p = e / l
+        o = p @ vp[cols]
+        dp = dop[r] @ vp[cols].T
+        ds = p * (dp - (dop[r] * o).sum(axis=-1, keepdims=True))
+        if qb in qblocks:
+            i = qblocks.index(qb)
+            dq[i] = ds @ kp[cols] * scale
+            lse[i] = (mx + np.log(l))[:, 0]
+        for i, b in enumerate(kblocks):
+            pos = np.nonzero(kept == b)[0]
+            if pos.size:
+                c = slice(int(pos[0]) * N, (int(pos[0]) + 1) * N)
+                dk[i] += ds[:, c].T @ qp[r] * scale
+                dv[i] += p[:, c].T @ dop[r]
+    return dq, dk, dv, lse
+
+
 def attention_backward_head(q, k, v, do, T, Hh, Ww, P, N, mask):
     """One head in natural order: fractal flatten, masked_attention_backward,
     inverse flatten. q, k, v, do: [S, d]. Returns (dq, dk, dv, lse) float64."""

@@ -83,3 +83,31 @@ def test_backward_matches_oracle(w, out_fp32):
             print(f"{w.name} fp32={out_fp32} head {bh} {name}: max {mx:.2e} mean {mean:.2e}")
             assert mx <= REL_MAX[out_fp32], (name, bh, mx)
             assert mean <= REL_MEAN[out_fp32], (name, bh, mean)
+
+
+def test_backward_full_size_sampled_blocks():
+    # HunyuanVideo-like grid (126,720 tokens, nb = 1980), two heads, bf16 as in
+    # the benchmark: dQ and the log-sum-exp of three q-blocks and dK, dV of
+    # three k-blocks per head, from the oracle's per-block form.
+    w = W.HUNYUAN.with_(name="hunyuan_1x2x126720x128", H=2)
+    dq, dk, dv, lse, mask = gpu_grads(w, False)
+    q, k, v = (x.reshape(w.BH, w.S, w.d) for x in W.make_inputs(w))
+    g = W.make_output_grad(w).reshape(w.BH, w.S, w.d)
+    perm = oracle.fractal_order(w.T, w.Hh, w.Ww, w.block)
+    qbs, kbs = [0, 777, w.nb - 1], [1, 990, w.nb - 2]
+    N = w.N
+    for bh in range(w.BH):
+        qp, kp, vp, dop = (oracle.flatten(oracle.widen_bf16(x[bh]), perm) for x in (q, k, v, g))
+        rq, rk, rv, rl = oracle.masked_attention_backward_blocks(qp, kp, vp, dop, mask[bh], N,
+                                                                 qbs, kbs)
+        got_q, got_k, got_v = (oracle.flatten(x[bh], perm) for x in (dq, dk, dv))
+        got_l = oracle.flatten(lse[bh][:, None], perm)[:, 0]
+        for i, b in enumerate(qbs):
+            assert np.abs(got_l[b * N:(b + 1) * N] - rl[i]).max() < LSE_ABS
+        for name, got, ref, blocks in (("dq", got_q, rq, qbs), ("dk", got_k, rk, kbs),
+                                       ("dv", got_v, rv, kbs)):
+            sample = np.stack([got[b * N:(b + 1) * N] for b in blocks])
+            mx, mean = rel_errors(sample, ref)
+            print(f"{w.name} head {bh} {name}: max {mx:.2e} mean {mean:.2e}")
+            assert mx <= REL_MAX[False], (name, bh, mx)
+            assert mean <= REL_MEAN[False], (name, bh, mean)

@@ -571,6 +571,26 @@ def test_backward_dense_is_torch_autograd():
     pin_backward_dense_is_torch_autograd()
 
 
+def test_backward_block_rows_match_full():
+    # The per-block form (used for full-size samples) against the full form,
+    # itself pinned by finite differences and autograd above.
+    rng = np.random.default_rng(53)
+    S, d, N = 512, 8, 64
+    nb = S // N
+    qp, kp, vp, dop = (rng.standard_normal((S, d)) for _ in range(4))
+    mask = rng.random((nb, nb)) < 0.4
+    mask[np.arange(nb), np.arange(nb)] = True
+    dq, dk, dv, lse = oracle.masked_attention_backward(qp, kp, vp, dop, mask, N)
+    qbs, kbs = [5, 0, 7], [3, 6]
+    bq, bk, bv, bl = oracle.masked_attention_backward_blocks(qp, kp, vp, dop, mask, N, qbs, kbs)
+    for i, b in enumerate(qbs):
+        assert np.abs(bq[i] - dq[b * N:(b + 1) * N]).max() < 1e-12
+        assert np.abs(bl[i] - lse[b * N:(b + 1) * N]).max() < 1e-12
+    for i, b in enumerate(kbs):
+        assert np.abs(bk[i] - dk[b * N:(b + 1) * N]).max() < 1e-12
+        assert np.abs(bv[i] - dv[b * N:(b + 1) * N]).max() < 1e-12
+
+
 def test_backward_uniform_rows():
     pin_backward_uniform_rows()
 
