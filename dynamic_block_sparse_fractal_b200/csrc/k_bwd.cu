@@ -144,23 +144,27 @@ cudaError_t launch_dq_convert(const float* dq_acc, void* dq, int out_fp32, const
 
 namespace {
 
-constexpr int kBThreads = 192;        // warp 0 TMA, warp 1 MMA, warps 2-5 rows
+constexpr int kBThreads = 320;        // warp 0 TMA, warp 1 MMA, warps 2-9 rows
 constexpr int kBChunk = 128 * 128;    // 128 rows x 128 B (64 bf16 channels)
-// TMEM columns: dV and dK accumulators (fp32, one key per lane); S^T, then P
-// (bf16 pairs, in place), then dQ (fp32, one query row per lane); dP^T, then
-// dS (bf16 pairs, in place).
+// TMEM columns: dV and dK accumulators (fp32, one key per lane); S^T, then P;
+// dP^T, then dS, then dQ (fp32, one query row per lane). Each row warpgroup
+// owns 64 columns of S^T and of dP^T (its q-block) and packs its P / dS
+// (bf16 pairs) into the first 32 of them, so the two never write columns the
+// other still reads; the MMAs read P and dS as two K = 64 halves.
 constexpr uint32_t kColDV = 0, kColDK = 128, kColS = 256, kColDP = 384;
+constexpr int kBMaxEntries = 2880;  // the most blocks a head may have
 
 template <int D>
 struct __align__(1024) BwdSmem {
   uint8_t k[D / 64][kBChunk];     // key tile: two k-blocks, 64 keys each
   uint8_t v[D / 64][kBChunk];
-  uint8_t q[D / 64][kBChunk];     // the step's query rows: two q-blocks
+  uint8_t q[2][D / 64][kBChunk];  // the step's query rows (two q-blocks), two slots
   uint8_t dout[D / 64][kBChunk];
   uint8_t ds[2][kBChunk];         // dS as the MN-major A of dQ = dS K: [64-query chunk][key][64 q]
-  float lse2[128], dsum[128];     // per query row of the step
-  uint64_t kv_full, q_full, q_empty, do_full, do_empty, st_full;
-  uint64_t s_full, p_full, dq_full, tmem_free, acc_full, drain;
+  float lse2[2][128], dsum[2][128];  // per query row of the step, two slots
+  int32_t ent[kBMaxEntries];      // the key tile's list (q-block | keep bits)
+  uint64_t kv_full, q_full[2], q_empty[2], do_full, do_empty, st_full[2], st_empty[2];
+  uint64_t s_full, dp_full, p_full, ds_full, dq_full, tmem_free, acc_full, drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -170,7 +174,8 @@ __device__ __forceinline__ void fail_b(uint32_t* status, int* abort, uint32_t bi
   *reinterpret_cast<volatile int*>(abort) = 1;
 }
 
-// 32 fp32 values -> row `row` of a [.][D] output, bf16 or fp32.
+// 32 fp32 values -> columns [col0, col0 + 32) of row `row` of a [.][D]
+// output, bf16 or fp32.
 template <int D>
 __device__ __forceinline__ void store_row32(void* out, size_t row, int col0, const float (&x)[32],
                                             int out_fp32) {
@@ -188,13 +193,26 @@ __device__ __forceinline__ void store_row32(void* out, size_t row, int col0, con
   }
 }
 
+// 64 packed bf16 pairs of this thread's key row: TMEM columns and the
+// 128-byte-swizzled dS row in shared memory (unit u of the row at u ^ (r & 7)).
+__device__ __forceinline__ void store_ds_row(uint8_t* row, int r, const uint32_t (&x)[32]) {
+#pragma unroll
+  for (int u = 0; u < 8; ++u)
+    *reinterpret_cast<uint4*>(row + ((u ^ (r & 7)) << 4)) =
+        make_uint4(x[4 * u], x[4 * u + 1], x[4 * u + 2], x[4 * u + 3]);
+}
+
 }  // namespace
 
 // One CTA per (key tile, bh): the key tile's K and V stay in shared memory;
-// each step takes the next two q-blocks of its list (S^T = K Q^T and
-// dP^T = V dO^T with the keys as the MMA's M), the row warps form P^T and
-// dS^T, then dV += P^T dO, dK += dS^T Q and dQ = dS K, whose rows are added
-// to the fp32 accumulator.
+// each step takes the next two q-blocks of its list. Per step:
+//   S^T = K Q^T        (keys as M)             -> row warps: P^T
+//   dP^T = V dO^T                               -> row warps: dS^T = P^T (dP^T - D)
+//   dV += P^T dO, dK += dS^T Q (A from TMEM), dQ = dS K (dS from shared
+//   memory), whose rows the row warps add to the fp32 accumulator.
+// The two row warpgroups take one q-block each (and half of dQ's columns);
+// the next step's S^T is issued right after this step's dQ, so it overlaps
+// the dQ read-out.
 template <int D>
 __global__ void __launch_bounds__(kBThreads, 1)
     bwd_kernel(const __grid_constant__ BwdArgs a, const Geometry g) {
@@ -207,20 +225,26 @@ __global__ void __launch_bounds__(kBThreads, 1)
   tile_blocks(g, tile, ka, kb);
   const size_t unit = size_t(bh) * g.ntile + tile;
   const int cnt = a.kcnt[unit];
-  const int32_t* ent = a.kidx + unit * g.nb;
   const int nsteps = (cnt + 1) / 2;
+  // the key tile's list, read once (every role walks it step by step)
+  for (int i = threadIdx.x; i < cnt; i += kBThreads) sm.ent[i] = a.kidx[unit * g.nb + i];
   if (threadIdx.x == 0) {
     sm.abort = 0;
     mbar_init(&sm.kv_full, 1);
-    mbar_init(&sm.q_full, 1);
-    mbar_init(&sm.q_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sm.q_full[s], 1);
+      mbar_init(&sm.q_empty[s], 1);
+      mbar_init(&sm.st_full[s], 1);
+      mbar_init(&sm.st_empty[s], 256);
+    }
     mbar_init(&sm.do_full, 1);
     mbar_init(&sm.do_empty, 1);
-    mbar_init(&sm.st_full, 1);
     mbar_init(&sm.s_full, 1);
-    mbar_init(&sm.p_full, 128);
+    mbar_init(&sm.dp_full, 1);
+    mbar_init(&sm.p_full, 256);
+    mbar_init(&sm.ds_full, 256);
     mbar_init(&sm.dq_full, 1);
-    mbar_init(&sm.tmem_free, 128);
+    mbar_init(&sm.tmem_free, 256);
     mbar_init(&sm.acc_full, 1);
     mbar_init(&sm.drain, 1);
     fence_barrier_init();
@@ -234,6 +258,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort = &sm.abort;
+  const int32_t* ent = sm.ent;
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA
@@ -254,26 +279,30 @@ __global__ void __launch_bounds__(kBThreads, 1)
                       t * g.pt, bh);
         }
       }
-      int last_st = -1, last_do = -1, last_q = -1;
+      int last_q = -1, last_do = -1, last_st = -1;
       for (int j = 0; j < nsteps; ++j) {
+        const int slot = j & 1;
         const bool two = 2 * j + 1 < cnt;
         const int nq = two ? 2 : 1;
         int blk[2];
         blk[0] = ent[2 * j] & kEntryBlockMask;
         blk[1] = two ? (ent[2 * j + 1] & kEntryBlockMask) : blk[0];
-        // statistics, once the row warps are done with the previous step's
-        if (j > 0 && !mbar_wait(&sm.p_full, (j - 1) & 1, abort)) {
+        // Q (two slots: loaded a step ahead)
+        if (j >= 2 && !mbar_wait(&sm.q_empty[slot], ((j >> 1) - 1) & 1, abort)) {
           fail_b(a.status, &sm.abort, kDevErrTimeoutLoad);
           break;
         }
-        mbar_arrive_expect_tx(&sm.st_full, uint32_t(nq) * 2u * 256u);
+        mbar_arrive_expect_tx(&sm.q_full[slot], uint32_t(nq) * 64u * D * 2u);
         for (int x = 0; x < nq; ++x) {
-          const size_t off = size_t(bh) * g.S + size_t(blk[x]) * 64;
-          bulk_load(&sm.lse2[64 * x], a.lse2 + off, 256u, &sm.st_full);
-          bulk_load(&sm.dsum[64 * x], a.dsum + off, 256u, &sm.st_full);
+          int t, hp, wp;
+          block_coords(g, blk[x], t, hp, wp);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_5d(&sm.q[slot][c][x * 8192], &a.map_q, &sm.q_full[slot], c * 64, wp * g.pw,
+                        hp * g.ph, t * g.pt, bh);
         }
-        last_st = j;
-        if (j > 0 && !mbar_wait(&sm.do_empty, (j - 1) & 1, abort)) {
+        last_q = j;
+        // dO (one slot: free once dV's MMA of the previous step is done)
+        if (j >= 1 && !mbar_wait(&sm.do_empty, (j - 1) & 1, abort)) {
           fail_b(a.status, &sm.abort, kDevErrTimeoutLoad);
           break;
         }
@@ -286,29 +315,30 @@ __global__ void __launch_bounds__(kBThreads, 1)
                         hp * g.ph, t * g.pt, bh);
         }
         last_do = j;
-        if (j > 0 && !mbar_wait(&sm.q_empty, (j - 1) & 1, abort)) {
+        // row statistics (two slots)
+        if (j >= 2 && !mbar_wait(&sm.st_empty[slot], ((j >> 1) - 1) & 1, abort)) {
           fail_b(a.status, &sm.abort, kDevErrTimeoutLoad);
           break;
         }
-        mbar_arrive_expect_tx(&sm.q_full, uint32_t(nq) * 64u * D * 2u);
+        mbar_arrive_expect_tx(&sm.st_full[slot], uint32_t(nq) * 2u * 256u);
         for (int x = 0; x < nq; ++x) {
-          int t, hp, wp;
-          block_coords(g, blk[x], t, hp, wp);
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_5d(&sm.q[c][x * 8192], &a.map_q, &sm.q_full, c * 64, wp * g.pw, hp * g.ph,
-                        t * g.pt, bh);
+          const size_t off = size_t(bh) * g.S + size_t(blk[x]) * 64;
+          bulk_load(&sm.lse2[slot][64 * x], a.lse2 + off, 256u, &sm.st_full[slot]);
+          bulk_load(&sm.dsum[slot][64 * x], a.dsum + off, 256u, &sm.st_full[slot]);
         }
-        last_q = j;
+        last_st = j;
         if (*abort) break;
       }
       if (*abort) {
         // let this thread's copies land before the CTA can exit (time-bounded,
-        // ignoring the abort flag)
+        // ignoring the abort flag); at most the last use of each slot is open
         int never = 0;
         mbar_wait(&sm.kv_full, 0, &never);
-        if (last_st >= 0) mbar_wait(&sm.st_full, last_st & 1, &never);
+        for (int jj = last_q; jj >= 0 && jj > last_q - 2; --jj)
+          mbar_wait(&sm.q_full[jj & 1], (jj >> 1) & 1, &never);
         if (last_do >= 0) mbar_wait(&sm.do_full, last_do & 1, &never);
-        if (last_q >= 0) mbar_wait(&sm.q_full, last_q & 1, &never);
+        for (int jj = last_st; jj >= 0 && jj > last_st - 2; --jj)
+          mbar_wait(&sm.st_full[jj & 1], (jj >> 1) & 1, &never);
       }
     }
   } else if (warp == 1) {
@@ -318,52 +348,62 @@ __global__ void __launch_bounds__(kBThreads, 1)
       const uint32_t id_s1 = idesc_bf16_f32(128, 64, 0, 0);
       const uint32_t id_acc = idesc_bf16_f32(128, D, 0, 1);  // A from TMEM, B MN-major
       const uint32_t id_dq = idesc_bf16_f32(128, D, 1, 1);   // A and B MN-major
+      constexpr uint32_t kSlot = (D / 64) * kBChunk / 16;    // a Q slot, descriptor units
+      constexpr uint64_t kHalfRows = 64 * 128 / 16;          // 64 rows of an MN-major tile
       const uint64_t kd = sw128_desc(smem_u32(&sm.k[0][0]), 16, 1024);
       const uint64_t vd = sw128_desc(smem_u32(&sm.v[0][0]), 16, 1024);
-      const uint64_t qd = sw128_desc(smem_u32(&sm.q[0][0]), 16, 1024);
+      const uint64_t qd0 = sw128_desc(smem_u32(&sm.q[0][0][0]), 16, 1024);
       const uint64_t dod = sw128_desc(smem_u32(&sm.dout[0][0]), 16, 1024);
-      const uint64_t q_mn = sw128_desc(smem_u32(&sm.q[0][0]), kBChunk, 1024);
+      const uint64_t q_mn0 = sw128_desc(smem_u32(&sm.q[0][0][0]), kBChunk, 1024);
       const uint64_t do_mn = sw128_desc(smem_u32(&sm.dout[0][0]), kBChunk, 1024);
       const uint64_t k_mn = sw128_desc(smem_u32(&sm.k[0][0]), kBChunk, 1024);
       const uint64_t ds_mn = sw128_desc(smem_u32(&sm.ds[0][0]), kBChunk, 1024);
       bool ok = mbar_wait(&sm.kv_full, 0, abort);
       for (int j = 0; ok && j < nsteps; ++j) {
+        const int slot = j & 1;
         const bool two = 2 * j + 1 < cnt;
-        ok = mbar_wait(&sm.q_full, j & 1, abort) && mbar_wait(&sm.do_full, j & 1, abort) &&
-             (j == 0 || mbar_wait(&sm.tmem_free, (j - 1) & 1, abort));
+        const uint32_t ids = two ? id_s2 : id_s1;
+        const uint64_t qd = qd0 + uint64_t(slot) * kSlot;
+        // S^T = K Q^T
+        ok = mbar_wait(&sm.q_full[slot], (j >> 1) & 1, abort);
         if (!ok) break;
         tc_fence_after_sync();
-        const uint32_t ids = two ? id_s2 : id_s1;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (uint32_t(kk >> 2) * kBChunk + uint32_t(kk & 3) * 32u) >> 4;
           mma_ss(tmem + kColS, kd + off, qd + off, ids, kk > 0);
         }
+        mma_commit(&sm.s_full);
+        // dP^T = V dO^T, once the previous step's dQ has left TMEM
+        ok = mbar_wait(&sm.do_full, j & 1, abort) &&
+             (j == 0 || mbar_wait(&sm.tmem_free, (j - 1) & 1, abort));
+        if (!ok) break;
+        tc_fence_after_sync();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (uint32_t(kk >> 2) * kBChunk + uint32_t(kk & 3) * 32u) >> 4;
           mma_ss(tmem + kColDP, vd + off, dod + off, ids, kk > 0);
         }
-        mma_commit(&sm.s_full);
+        mma_commit(&sm.dp_full);
+        // dV += P^T dO over the step's query rows (K = 128 or 64)
         ok = mbar_wait(&sm.p_full, j & 1, abort);
         if (!ok) break;
         tc_fence_after_sync();
-        // dV += P^T dO and dK += dS^T Q over the step's query rows (K = 128
-        // or 64); each commit frees the tile it was the last reader of
-        if (two)
-          mma_ts_k<8>(tmem + kColDV, tmem + kColS, do_mn, id_acc, j > 0 ? 1u : 0u);
-        else
-          mma_ts_k<4>(tmem + kColDV, tmem + kColS, do_mn, id_acc, j > 0 ? 1u : 0u);
+        // (the second q-block's P sits 64 columns on; its dO rows 64 rows on)
+        mma_ts_k<4>(tmem + kColDV, tmem + kColS, do_mn, id_acc, j > 0 ? 1u : 0u);
+        if (two) mma_ts_k<4>(tmem + kColDV, tmem + kColS + 64u, do_mn + kHalfRows, id_acc, 1u);
         mma_commit(&sm.do_empty);
-        if (two)
-          mma_ts_k<8>(tmem + kColDK, tmem + kColDP, q_mn, id_acc, j > 0 ? 1u : 0u);
-        else
-          mma_ts_k<4>(tmem + kColDK, tmem + kColDP, q_mn, id_acc, j > 0 ? 1u : 0u);
-        mma_commit(&sm.q_empty);
-        // dQ = dS K: the 128 query rows as M, the 128 keys as K
+        // dK += dS^T Q, then dQ = dS K over the dS columns (read just before)
+        ok = mbar_wait(&sm.ds_full, j & 1, abort);
+        if (!ok) break;
+        tc_fence_after_sync();
+        const uint64_t q_mn = q_mn0 + uint64_t(slot) * kSlot;
+        mma_ts_k<4>(tmem + kColDK, tmem + kColDP, q_mn, id_acc, j > 0 ? 1u : 0u);
+        if (two) mma_ts_k<4>(tmem + kColDK, tmem + kColDP + 64u, q_mn + kHalfRows, id_acc, 1u);
+        mma_commit(&sm.q_empty[slot]);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + kColS, ds_mn + uint64_t(kk) * 128u, k_mn + uint64_t(kk) * 128u, id_dq,
+          mma_ss(tmem + kColDP, ds_mn + uint64_t(kk) * 128u, k_mn + uint64_t(kk) * 128u, id_dq,
                  kk > 0);
         mma_commit(&sm.dq_full);
       }
@@ -378,94 +418,129 @@ __global__ void __launch_bounds__(kBThreads, 1)
     }
   } else {
     // ---------------------------------------------------------------- rows
-    const int quad = warp & 3;
+    // warpgroup wg takes query columns [64 wg, 64 wg + 64) of S^T / dP^T (its
+    // q-block of the step) and dQ / dK / dV columns [D/2 wg, D/2 (wg + 1))
+    constexpr int DH = D / 2;
+    const int wg = (warp - 2) >> 2, quad = warp & 3;
     const int r = quad * 32 + lane;  // TMEM lane: a key in S^T, dP^T, dK, dV; a query row in dQ
     const uint32_t lane_base = tmem + (uint32_t(quad * 32) << 16);
     const int my_keep = r < 64 ? kEntryKeepA : kEntryKeepB;  // uniform across the warp
     const float sl2 = a.scale_log2;
     bool ok = true;
     for (int j = 0; j < nsteps; ++j) {
+      const int slot = j & 1;
       const bool two = 2 * j + 1 < cnt;
       const int f0 = ent[2 * j], f1 = two ? ent[2 * j + 1] : 0;
+      const bool mine = wg == 0 || two;                       // this half has a q-block
+      const bool keep = mine && (((wg ? f1 : f0) & my_keep) != 0);  // uniform across the warp
+      const float* lse2 = &sm.lse2[slot][64 * wg];
+      const float* dsum = &sm.dsum[slot][64 * wg];
+      // ---- P^T = 2^(s log2(e)/sqrt(d) - lse2) on a kept (k-block, q-block) pair
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sm.s_full, j & 1, abort) &&
-                                       mbar_wait(&sm.st_full, j & 1, abort));
+                                       mbar_wait(&sm.st_full[slot], (j >> 1) & 1, abort));
       if (!ok) break;
       tc_fence_after_sync();
-      // P^T = 2^(s log2(e)/sqrt(d) - lse2) on kept (k-block, q-block) pairs,
-      // dS^T = P^T * (dP^T - D); 32 query columns per chunk
-      for (int c = 0; c < (two ? 4 : 2); ++c) {
-        const bool keep = (((c < 2) ? f0 : f1) & my_keep) != 0;
-        uint32_t pk[16], dk[16];
-        if (keep) {
-          uint32_t sv[32], dp[32];
-          tmem_ld32(lane_base + kColS + 32u * c, sv);
-          tmem_ld32(lane_base + kColDP + 32u * c, dp);
+      float p[64];
+      uint32_t pk[32];
+      const uint32_t s_col = lane_base + kColS + 64u * wg;    // this half's S^T, then P
+      const uint32_t dp_col = lane_base + kColDP + 64u * wg;  // this half's dP^T, then dS
+      if (keep) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t sv[32];
+          tmem_ld32(s_col + 32u * c, sv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            p[32 * c + i] = ex2_approx(fmaf(__uint_as_float(sv[i]), sl2, -lse2[32 * c + i]));
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(p[2 * i], p[2 * i + 1]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) pk[i] = 0u;
+      }
+      if (mine) tmem_st32(s_col, pk);
+      tmem_wait_st();
+      tc_fence_before_sync();
+      // relaxed: the stores above are complete, and the previous step's dQ
+      // reductions need not be
+      mbar_arrive_relaxed(&sm.p_full);
+      // ---- dS^T = P^T (dP^T - D)
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sm.dp_full, j & 1, abort));
+      if (!ok) break;
+      tc_fence_after_sync();
+      if (keep) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t dp[32];
+          tmem_ld32(dp_col + 32u * c, dp);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const int col = 32 * c + 2 * i;
-            const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * i]), sl2, -sm.lse2[col]));
-            const float p1 =
-                ex2_approx(fmaf(__uint_as_float(sv[2 * i + 1]), sl2, -sm.lse2[col + 1]));
-            const float d0 = p0 * (__uint_as_float(dp[2 * i]) - sm.dsum[col]);
-            const float d1 = p1 * (__uint_as_float(dp[2 * i + 1]) - sm.dsum[col + 1]);
-            pk[i] = pack_bf16x2(p0, p1);
-            dk[i] = pack_bf16x2(d0, d1);
+            const int k2 = 32 * c + 2 * i;
+            pk[16 * c + i] = pack_bf16x2(p[k2] * (__uint_as_float(dp[2 * i]) - dsum[k2]),
+                                         p[k2 + 1] * (__uint_as_float(dp[2 * i + 1]) - dsum[k2 + 1]));
           }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) pk[i] = dk[i] = 0u;
         }
-        tmem_st16(lane_base + kColS + 16u * c, pk);
-        tmem_st16(lane_base + kColDP + 16u * c, dk);
-        // this key's row of dS in the 128-byte-swizzled MN-major layout:
-        // 16-byte unit u of the row sits at unit u ^ (r & 7)
-        uint8_t* row = &sm.ds[c >> 1][r * 128];
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const int u = ((c & 1) << 2) + w;
-          *reinterpret_cast<uint4*>(row + ((u ^ (r & 7)) << 4)) =
-              make_uint4(dk[4 * w], dk[4 * w + 1], dk[4 * w + 2], dk[4 * w + 3]);
-        }
-      }
-      if (!two) {
-        // dQ's MMA reads all 128 query rows of dS: zero the absent q-block's
-        uint8_t* row = &sm.ds[1][r * 128];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) *reinterpret_cast<uint4*>(row + (u << 4)) = make_uint4(0, 0, 0, 0);
-      }
+      }  // otherwise pk is still all zero
+      if (mine) tmem_st32(dp_col, pk);
+      // dQ's MMA reads all 128 query rows of dS: an absent q-block's are zero
+      store_ds_row(&sm.ds[wg][r * 128], r, pk);
       fence_proxy_async_smem();
       tmem_wait_st();
       tc_fence_before_sync();
-      mbar_arrive(&sm.p_full);
-      // dQ rows (one query row per lane) -> the fp32 accumulator
+      mbar_arrive(&sm.ds_full);
+      mbar_arrive(&sm.st_empty[slot]);
+      // ---- dQ rows (one query row per lane, this half's columns) -> the fp32
+      // accumulator by vector reductions. Each warp turns its 32 rows x 32
+      // columns around in a 4 KB staging tile (in the dS buffer, free from
+      // dQ's MMA until the next step's dP^T, which waits for every thread's
+      // TMEM release below), so that one reduction instruction covers four
+      // whole 128-byte row segments: full-sector L2 operations. TMEM is
+      // released with a relaxed arrive once read (tcgen05.wait::ld), so the
+      // reductions in flight do not hold the next step's MMAs back.
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sm.dq_full, j & 1, abort));
       if (!ok) break;
       tc_fence_after_sync();
       const int h = r >> 6;  // uniform across the warp
       if (h == 0 || two) {
         const int blk = (h ? f1 : f0) & kEntryBlockMask;
-        float* dst = a.dq_acc + (size_t(bh) * g.S + block_row_token(g, blk, r & 63)) * D;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        const unsigned long long dst = reinterpret_cast<unsigned long long>(
+            a.dq_acc + (size_t(bh) * g.S + block_row_token(g, blk, r & 63)) * D + DH * wg);
+        uint8_t* stage = &sm.ds[0][0] + (warp - 2) * 4096;
+        for (int c = 0; c < DH / 32; ++c) {
           uint32_t o[32];
-          tmem_ld32(lane_base + kColS + 32u * c, o);
+          tmem_ld32(lane_base + kColDP + uint32_t(DH * wg + 32 * c), o);
           tmem_wait_ld();
+          // this lane's row segment, 16-byte units swizzled by row
 #pragma unroll
-          for (int v = 0; v < 8; ++v)
-            red_add_f32x4(dst + 32 * c + 4 * v, __uint_as_float(o[4 * v]) * a.scale,
-                          __uint_as_float(o[4 * v + 1]) * a.scale,
-                          __uint_as_float(o[4 * v + 2]) * a.scale,
-                          __uint_as_float(o[4 * v + 3]) * a.scale);
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<float4*>(stage + lane * 128 + ((u ^ (lane & 7)) << 4)) =
+                make_float4(__uint_as_float(o[4 * u]) * a.scale,
+                            __uint_as_float(o[4 * u + 1]) * a.scale,
+                            __uint_as_float(o[4 * u + 2]) * a.scale,
+                            __uint_as_float(o[4 * u + 3]) * a.scale);
+          __syncwarp();
+          // 8 lanes per row segment, 4 rows per instruction
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int row = 4 * i + (lane >> 3), u = lane & 7;
+            const float4 x =
+                *reinterpret_cast<const float4*>(stage + row * 128 + ((u ^ (row & 7)) << 4));
+            float* p = reinterpret_cast<float*>(__shfl_sync(0xFFFFFFFFu, dst, row));
+            red_add_f32x4(p + 32 * c + 4 * u, x.x, x.y, x.z, x.w);
+          }
+          __syncwarp();  // the tile is reused by the next segment
         }
       }
       tc_fence_before_sync();
-      mbar_arrive(&sm.tmem_free);
+      mbar_arrive_relaxed(&sm.tmem_free);
     }
     if (!ok) {
       fail_b(a.status, &sm.abort, kDevErrTimeoutSoftmax);
     } else if (r < 64 || kb >= 0) {  // uniform across the warp
-      // dK (scaled) and dV rows of this key to its natural position
+      // dK (scaled) and dV of this key, this half's columns, to its natural position
       const bool acc = nsteps == 0 || __all_sync(0xFFFFFFFFu, mbar_wait(&sm.acc_full, 0, abort));
       if (!acc) {
         fail_b(a.status, &sm.abort, kDevErrTimeoutSoftmax);
@@ -475,11 +550,12 @@ __global__ void __launch_bounds__(kBThreads, 1)
         for (int which = 0; which < 2; ++which) {
           const float mul = which ? a.scale : 1.0f;
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < DH / 32; ++c) {
+            const int col = DH * wg + 32 * c;
             float x[32];
             if (nsteps > 0) {
               uint32_t o[32];
-              tmem_ld32(lane_base + (which ? kColDK : kColDV) + 32u * c, o);
+              tmem_ld32(lane_base + (which ? kColDK : kColDV) + uint32_t(col), o);
               tmem_wait_ld();
 #pragma unroll
               for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(o[i]) * mul;
@@ -487,7 +563,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
 #pragma unroll
               for (int i = 0; i < 32; ++i) x[i] = 0.f;
             }
-            store_row32<D>(which ? a.dk : a.dv, row, 32 * c, x, a.out_fp32);
+            store_row32<D>(which ? a.dk : a.dv, row, col, x, a.out_fp32);
           }
         }
       }
