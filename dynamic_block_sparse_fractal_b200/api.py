@@ -30,7 +30,8 @@ SYMBOLS = (
     "sparse_attn_workspace_size_heads", "sparse_attn_plan_heads", "sparse_attn_fwd_heads",
     "sparse_attn_check_heads", "sparse_attn_heads_run", "sparse_attn_block_heatmap",
     "sparse_attn_block_heatmap_scratch_size", "sparse_attn_fwd_lse",
-    "sparse_attn_bwd_scratch_size", "sparse_attn_bwd",
+    "sparse_attn_bwd_scratch_size", "sparse_attn_bwd", "sparse_attn_graph_create",
+    "sparse_attn_graph_launch", "sparse_attn_graph_destroy",
 )
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -355,6 +356,42 @@ def heads_runs(desc: SaDesc, tiles):
         _ok(st, "heads_run")
         out.append((sub, h0.value, off.value, nbytes.value))
         i += 1
+
+
+class AttentionGraph:
+    """Plan (optional) + forward captured once as a CUDA graph on fixed
+    tensors; ``launch`` replays the whole path with one launch on whatever
+    the tensors then hold. See include/sparse_attn.h."""
+
+    def __init__(self, desc: SaDesc, q, k, v, workspace, out, with_plan: bool = True):
+        _check_qkv(desc, q, k, v)
+        want = torch.float32 if desc.out_fp32 else torch.bfloat16
+        if out.dtype != want or out.shape != q.shape or not out.is_contiguous():
+            raise ValueError(f"out must be a contiguous {want} tensor shaped like q")
+        self.desc = desc
+        self._buffers = (q, k, v, workspace, out)  # the graph holds their addresses
+        h = ctypes.c_void_p()
+        _ok(lib().sparse_attn_graph_create(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v),
+                                           _ptr(workspace), ctypes.c_size_t(workspace.numel()),
+                                           _ptr(out), int(bool(with_plan)), ctypes.byref(h)),
+            "graph_create")
+        self._h = h
+
+    def launch(self, stream=None) -> None:
+        if not self._h:
+            raise ValueError("graph already destroyed")
+        _ok(lib().sparse_attn_graph_launch(self._h, _stream(stream)), "graph_launch")
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            lib().sparse_attn_graph_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 class NablaAttention:

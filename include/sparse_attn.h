@@ -228,6 +228,30 @@ sa_status sparse_attn_check_heads(const sa_desc* desc, const int* tiles, const v
 sa_status sparse_attn_heads_run(const sa_desc* desc, const int* tiles, int run, sa_desc* sub,
                                 int* head0, size_t* ws_offset, size_t* ws_bytes);
 
+/* ---- Whole path as one launch (CUDA graph) --------------------------------
+ * Plan reuse across calls and steps is the pages' recurring economy (the
+ * SVG2 page caches centroids across denoising steps, the TRA page reuses its
+ * masks, the Veda page caches tile scores over time). These calls capture
+ * sparse_attn_plan (with_plan = 1) and sparse_attn_fwd on fixed buffers into
+ * a CUDA graph once; each replay runs the whole path with a single launch on
+ * whatever the buffers then hold. with_plan = 0 captures only the forward,
+ * reusing the plan already in the workspace. The graph object is the one
+ * thing the library allocates (host memory and the driver's graph), owned by
+ * the caller until sparse_attn_graph_destroy. Arguments are validated as by
+ * the captured calls; nothing runs during creation. */
+typedef struct sa_graph sa_graph;
+
+sa_status sparse_attn_graph_create(const sa_desc* desc, const void* q, const void* k,
+                                   const void* v, void* workspace, size_t ws_bytes, void* out,
+                                   int with_plan, sa_graph** graph);
+
+/* One replay on `stream` (asynchronous; sparse_attn_check reports device
+ * timeouts as for the captured calls). */
+sa_status sparse_attn_graph_launch(sa_graph* graph, void* stream);
+
+/* Releases the graph (NULL is a no-op). */
+sa_status sparse_attn_graph_destroy(sa_graph* graph);
+
 /* ---- Gradients (training use of the mask) ---------------------------------
  * The NABLA page uses the same block mask when training a DiT ("Risultati
  * Sperimentali"), which needs the gradients of the masked attention. With

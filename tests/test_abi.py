@@ -88,6 +88,16 @@ def test_entry_points_reject_before_launch():
     assert heat_call(need, FAKE, None, scr) == api.SA_ERR_INVALID_ARG  # no scratch
     assert heat_call(need - 1, FAKE, FAKE, scr) == api.SA_ERR_WORKSPACE
     assert heat_call(need, FAKE, FAKE, scr - 1) == api.SA_ERR_WORKSPACE
+    h = ctypes.c_void_p()
+    assert L.sparse_attn_graph_create(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, sz(need), FAKE, 1,
+                                      None) == api.SA_ERR_INVALID_ARG  # nowhere to put it
+    assert L.sparse_attn_graph_create(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, sz(need), FAKE, 2,
+                                      ctypes.byref(h)) == api.SA_ERR_INVALID_ARG
+    bad = api.make_desc(1, 1, 4, 8, 8, 96, 0.1)  # d = 96: rejected before any capture
+    assert L.sparse_attn_graph_create(ctypes.byref(bad), FAKE, FAKE, FAKE, FAKE, sz(need), FAKE, 1,
+                                      ctypes.byref(h)) == api.SA_ERR_UNSUPPORTED
+    assert L.sparse_attn_graph_launch(None, None) == api.SA_ERR_INVALID_ARG
+    assert L.sparse_attn_graph_destroy(None) == api.SA_OK
 
 
 @pytest.mark.parametrize("T,Hh,Ww", [(4, 8, 8), (33, 48, 80), (21, 32, 56), (3, 8, 24), (1, 16, 8)])
