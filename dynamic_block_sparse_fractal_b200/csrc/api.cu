@@ -220,6 +220,7 @@ sa_status sparse_attn_bwd(const sa_desc* desc, const void* q, const void* k, con
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)g.d));
   a.scale = (float)(1.0 / std::sqrt((double)g.d));
   a.out_fp32 = desc->out_fp32;
+  a.debug_flags = desc->debug_flags;
   cudaError_t e = cudaMemsetAsync(a.dq_acc, 0, sizeof(float) * size_t(g.BH) * g.S * g.d, s);
   if (e == cudaSuccess)
     e = launch_bwd_prep(out, dout, lse, at<float>(scratch, b.lse2), at<float>(scratch, b.dsum),
@@ -262,6 +263,7 @@ sa_status sparse_attn_block_heatmap(const sa_desc* desc, const void* q, const vo
   a.scratch = static_cast<float*>(scratch);
   a.status = at<uint32_t>(workspace, w.status);
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)g.d));
+  a.debug_flags = desc->debug_flags;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(a.status, 0, sizeof(uint32_t), s) != cudaSuccess) return SA_ERR_CUDA;
   return cuda_status(launch_heat(a, g, s));

@@ -292,15 +292,16 @@ __global__ void __launch_bounds__(kBThreads, 1)
           fail_b(a.status, &sm.abort, kDevErrTimeoutLoad);
           break;
         }
-        mbar_arrive_expect_tx(&sm.q_full[slot], uint32_t(nq) * 64u * D * 2u);
-        for (int x = 0; x < nq; ++x) {
+        const bool stall = j == 0 && (a.debug_flags & SA_DEBUG_STALL_LOADER);  // test hook
+        if (!stall) mbar_arrive_expect_tx(&sm.q_full[slot], uint32_t(nq) * 64u * D * 2u);
+        for (int x = 0; x < nq && !stall; ++x) {
           int t, hp, wp;
           block_coords(g, blk[x], t, hp, wp);
           for (int c = 0; c < D / 64; ++c)
             tma_load_5d(&sm.q[slot][c][x * 8192], &a.map_q, &sm.q_full[slot], c * 64, wp * g.pw,
                         hp * g.ph, t * g.pt, bh);
         }
-        last_q = j;
+        if (!stall) last_q = j;
         // dO (one slot: free once dV's MMA of the previous step is done)
         if (j >= 1 && !mbar_wait(&sm.do_empty, (j - 1) & 1, abort)) {
           fail_b(a.status, &sm.abort, kDevErrTimeoutLoad);

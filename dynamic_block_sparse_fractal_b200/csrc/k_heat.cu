@@ -165,6 +165,7 @@ __global__ void __launch_bounds__(kHThreads, 1)
             ok = false;
             break;
           }
+          if (op == 0 && (a.debug_flags & SA_DEBUG_STALL_LOADER)) continue;  // test hook
           const int nblk = 2 * j + 1 < g.nb ? 2 : 1;
           mbar_arrive_expect_tx(&sm.full[s], uint32_t(nblk) * 64u * D * 2u);
           for (int e = 0; e < nblk; ++e) {

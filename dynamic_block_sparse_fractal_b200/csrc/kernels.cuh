@@ -70,6 +70,7 @@ struct HeatArgs {
   float* scratch;            // [heat_ctas(g)][nb][256]
   uint32_t* status;
   float scale_log2;  // log2(e) / sqrt(d)
+  int debug_flags;   // SA_DEBUG_STALL_LOADER: the first K load is never issued (test hook)
 };
 // Gradients of the block-sparse attention. Scratch (every region 256-byte
 // aligned): dq_acc fp32 [BH][S][d] natural order (zeroed, then reduced into),
@@ -105,6 +106,7 @@ struct BwdArgs {
   float scale_log2;  // log2(e) / sqrt(d)
   float scale;       // 1 / sqrt(d)
   int out_fp32;
+  int debug_flags;   // SA_DEBUG_STALL_LOADER: the first Q load is never issued (test hook)
 };
 // D = rowsum(dO * O) and lse * log2(e), both into fractal order (o: bf16 or
 // fp32 per o_fp32; do_: bf16; lse: natural-log row log-sum-exp, natural order).

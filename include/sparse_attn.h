@@ -273,7 +273,8 @@ sa_status sparse_attn_bwd_scratch_size(const sa_desc* desc, size_t* bytes);
 
 /* dq, dk, dv = gradients of sum(out * dout) with respect to q, k, v, over the
  * mask of the plan in `workspace` (made for the same desc; its status word
- * collects device timeouts, see sparse_attn_check). q, k, v: as for
+ * collects device timeouts, see sparse_attn_check, and keeps them until the
+ * next sparse_attn_plan clears it). q, k, v: as for
  * sparse_attn_fwd; out, lse: what sparse_attn_fwd_lse wrote for them (out
  * bf16, or fp32 if desc->out_fp32); dout: [B,H,S,d] bf16 (it is a
  * tensor-core operand). dq, dk, dv: [B,H,S,d], natural order, bf16 (fp32 if
@@ -287,7 +288,7 @@ sa_status sparse_attn_bwd(const sa_desc* desc, const void* q, const void* k, con
 
 /* ---- Block max-pooled attention map (mask diagnostics) -------------------
  * "Veda: Video Generation with Efficient Sparse Attention", section 2.1
- * ("Costruzione dell'Obiettivo"): the reference a block mask is judged
+ * ("Costruzione dell'Obiettivo"): the reference a block mask is measured
  * against is the full, unmasked attention P = softmax(Q K^T / sqrt(d)) of a
  * head, max-pooled over every N x N block:
  *   heat[bh][i][j] = max over q in block i, k in block j of P[q][k],

@@ -339,3 +339,35 @@ def test_per_head_shapes_match_oracle_head_by_head():
                                         w.thr, w.sta, mask=gm)
         res = parity.out_check(out_np[heads], ref, True)
         assert res["ok"], (tile, res)
+
+
+def test_heatmap_and_backward_timeouts_are_reported_and_context_survives():
+    # The same test hook in the map and gradient kernels: the first K (map) or
+    # Q (gradients) load is never issued, every wait on it runs out after its
+    # bound, the kernel records the status and drains; the next call is normal.
+    w = W.TINY
+    q, k, v = (to_dev(x, w) for x in host_inputs(w))
+    stall = api.desc_for(w, out_fp32=True, debug_flags=api.SA_DEBUG_STALL_LOADER)
+    desc = api.desc_for(w, out_fp32=True)
+    ws = api.alloc_workspace(desc)
+    api.plan(desc, q, k, ws)
+    api.block_heatmap(stall, q, k, ws)
+    assert api.check(stall, ws) == api.SA_ERR_DEVICE_TIMEOUT
+    heat = api.block_heatmap(desc, q, k, ws)
+    assert api.check(desc, ws) == api.SA_OK
+    qh, kh, _ = host_inputs(w)
+    for bh in range(w.BH):
+        ref = oracle.block_heatmap(qh[bh], kh[bh], w.T, w.Hh, w.Ww, w.block, w.N)
+        np.testing.assert_allclose(heat[bh].cpu().numpy(), ref, rtol=1e-3, atol=1e-9)
+    out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device="cuda")
+    api.fwd_lse(desc, q, k, v, ws, out, lse)
+    g = torch.randn(q.shape, device="cuda").to(torch.bfloat16)
+    api.bwd(stall, q, k, v, out, g, lse, ws)
+    assert api.check(stall, ws) == api.SA_ERR_DEVICE_TIMEOUT
+    api.plan(desc, q, k, ws)  # the status word is sticky until the next plan clears it
+    good = api.bwd(desc, q, k, v, out, g, lse, ws)
+    assert api.check(desc, ws) == api.SA_OK
+    again = api.bwd(desc, q, k, v, out, g, lse, ws)
+    for a, b in zip(good, again):  # fp32 reductions in any order: equal to rounding
+        assert torch.allclose(a, b, rtol=1e-5, atol=1e-6)
