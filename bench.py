@@ -1,7 +1,8 @@
 """Benchmark of the block-sparse video attention path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--no-cpu-baseline]
+                    [--workload NAME] [--heads H] [--no-cpu-baseline] [--no-heatmap]
+                    [--no-backward]
 
 One step = one pass of the whole hot path over one batch: sparse_attn_plan
 (block pooling, reduced map, CDF threshold, STA union, block lists) followed by
@@ -9,7 +10,10 @@ sparse_attn_fwd (block-sparse attention over the kept pairs, written back in
 natural token order). The metric is attention TFLOP/s counted on kept blocks
 only (4 * 64^2 * d per kept (q-block, k-block) pair), whole step; the JSON
 also carries the mask-build time, the attention kernel's own TFLOP/s and its
-fraction of the measured bf16 tensor peak.
+fraction of the measured bf16 tensor peak. Measured outside the timed step and
+reported beside it: the exact block max-pooled attention map (its kernel time
+and the mask's recall against it) and the gradients over the mask (one
+sparse_attn_bwd call).
 
 With N > 1 (launched by torch.distributed.run) every rank runs its own copy of
 the workload (heads are independent: weak scaling, no data-path collective);
@@ -453,7 +457,7 @@ def run_reference(args, w, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=None)
