@@ -416,5 +416,24 @@ class NablaAttention:
         self.plan(q, k, stream)
         return self.forward(q, k, v, out, stream)
 
+    def forward_lse(self, q, k, v, out=None, lse=None, stream=None):
+        """Forward over the current plan, also returning each row's log-sum-exp
+        (what ``backward`` needs): (out, lse)."""
+        if out is None:
+            out = torch.empty(q.shape, device=q.device,
+                              dtype=torch.float32 if self.desc.out_fp32 else torch.bfloat16)
+        if lse is None:
+            lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+        fwd_lse(self.desc, q, k, v, self.workspace, out, lse, stream)
+        return out, lse
+
+    def backward(self, q, k, v, out, dout, lse, stream=None):
+        """(dq, dk, dv) of sum(out * dout) over the current plan's mask."""
+        return bwd(self.desc, q, k, v, out, dout, lse, self.workspace, stream=stream)
+
+    def heatmap(self, q, k, stream=None):
+        """Exact block max-pooled full-attention map [B*H, nb, nb]."""
+        return block_heatmap(self.desc, q, k, self.workspace, stream=stream)
+
     def check(self, stream=None) -> int:
         return check(self.desc, self.workspace, stream)

@@ -111,3 +111,27 @@ def test_backward_full_size_sampled_blocks():
             print(f"{w.name} head {bh} {name}: max {mx:.2e} mean {mean:.2e}")
             assert mx <= REL_MAX[False], (name, bh, mx)
             assert mean <= REL_MEAN[False], (name, bh, mean)
+
+
+def test_nabla_attention_methods_match_functional_calls():
+    w = W.TINY
+    q, k, v = (to_dev(x) for x in W.make_inputs(w))
+    g = to_dev(W.make_output_grad(w))
+    attn = api.NablaAttention(w.B, w.H, w.T, w.Hh, w.Ww, w.d, w.thr, w.sta, out_fp32=True)
+    attn.plan(q, k)
+    out, lse = attn.forward_lse(q, k, v)
+    grads = attn.backward(q, k, v, out, g, lse)
+    heat = attn.heatmap(q, k)
+    assert attn.check() == api.SA_OK
+    desc = api.desc_for(w, out_fp32=True)
+    ws = api.alloc_workspace(desc)
+    api.plan(desc, q, k, ws)
+    out2 = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    lse2 = torch.empty(q.shape[:3], dtype=torch.float32, device="cuda")
+    api.fwd_lse(desc, q, k, v, ws, out2, lse2)
+    grads2 = api.bwd(desc, q, k, v, out2, g, lse2, ws)
+    heat2 = api.block_heatmap(desc, q, k, ws)
+    assert api.check(desc, ws) == api.SA_OK
+    assert torch.equal(out, out2) and torch.equal(lse, lse2) and torch.equal(heat, heat2)
+    for a, b in zip(grads, grads2):  # fp32 reductions in any order: equal to rounding
+        assert torch.allclose(a, b, rtol=1e-5, atol=1e-6)
