@@ -304,7 +304,13 @@ def run_ours(args, w, rank, world):
     ms_step = total_ms / args.steps
     fwd_avg = statistics.mean(fwd_ms)
     attn_tflops = kept_flops / (fwd_avg * 1e-3) / 1e12
-    peak = float(peaks["bf16_tflops"])
+    # The denominator follows the timing: the burst GEMM figure for a short
+    # timed region, the sustained (power-capped) one when the kernel runs for
+    # about a second or more under load, as the default 40 steps do.
+    long_run = total_ms >= 500.0 and "bf16_tflops_sustained" in peaks
+    peak = float(peaks["bf16_tflops_sustained"] if long_run else peaks["bf16_tflops"])
+    other = float(peaks["bf16_tflops"]) if long_run else (
+        float(peaks["bf16_tflops_sustained"]) if "bf16_tflops_sustained" in peaks else None)
     line = {
         "metric": METRIC, "value": round(aggregate_tflops(world, kept_flops, ms_step), 2),
         "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -322,10 +328,11 @@ def run_ours(args, w, rank, world):
         "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 2), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(attn_tflops / peak, 4),
                      "traffic": attn_traffic(w), "kernel": "sa::attn_kernel<128>",
-                     "peak_source": f"{src} bf16 burst",
-                     # context: the same against the power-capped sustained GEMM figure
-                     "frac_of_sustained": (round(attn_tflops / float(peaks["bf16_tflops_sustained"]), 4)
-                                           if "bf16_tflops_sustained" in peaks else None)},
+                     "peak_source": f"{src} bf16 {'sustained' if long_run else 'burst'} "
+                                    f"(timed region {total_ms / 1e3:.2f} s)",
+                     # context: the same rate against the other measured figure
+                     ("frac_of_burst" if long_run else "frac_of_sustained"):
+                         round(attn_tflops / other, 4) if other else None},
         "e2e": {"value": round(aggregate_tflops(world, kept_flops, e2e_ms), 2), "unit": UNIT,
                 "ms_per_step": round(e2e_ms, 3), "steps": e2e_steps,
                 "overlap": "double-buffered: H2D of step i+1 and D2H of step i-1 overlap step i",
