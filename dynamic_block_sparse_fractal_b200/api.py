@@ -31,7 +31,9 @@ SYMBOLS = (
     "sparse_attn_check_heads", "sparse_attn_heads_run", "sparse_attn_block_heatmap",
     "sparse_attn_block_heatmap_scratch_size", "sparse_attn_fwd_lse",
     "sparse_attn_bwd_scratch_size", "sparse_attn_bwd", "sparse_attn_graph_create",
-    "sparse_attn_graph_launch", "sparse_attn_graph_destroy",
+    "sparse_attn_graph_launch", "sparse_attn_graph_destroy", "sparse_attn_fwd_lse_heads",
+    "sparse_attn_bwd_scratch_size_heads", "sparse_attn_bwd_heads",
+    "sparse_attn_block_heatmap_scratch_size_heads", "sparse_attn_block_heatmap_heads",
 )
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -340,6 +342,53 @@ def fwd_heads(desc: SaDesc, tiles, q, k, v, workspace, out, stream=None):
 def check_heads(desc: SaDesc, tiles, workspace, stream=None) -> int:
     return lib().sparse_attn_check_heads(ctypes.byref(desc), _tiles_array(tiles),
                                          _ptr(workspace), workspace.numel(), _stream(stream))
+
+
+def fwd_lse_heads(desc: SaDesc, tiles, q, k, v, workspace, out, lse, stream=None):
+    _check_qkv(desc, q, k, v)
+    if lse.dtype != torch.float32 or tuple(lse.shape) != tuple(q.shape[:3]) or \
+            not lse.is_contiguous():
+        raise ValueError(f"lse must be a contiguous float32 tensor of shape {tuple(q.shape[:3])}")
+    _ok(lib().sparse_attn_fwd_lse_heads(ctypes.byref(desc), _tiles_array(tiles), _ptr(q), _ptr(k),
+                                        _ptr(v), _ptr(workspace),
+                                        ctypes.c_size_t(workspace.numel()), _ptr(out), _ptr(lse),
+                                        _stream(stream)), "fwd_lse_heads")
+    return out
+
+
+def bwd_heads(desc: SaDesc, tiles, q, k, v, out, dout, lse, workspace, stream=None):
+    """(dq, dk, dv) with per-head block shapes; see include/sparse_attn.h."""
+    _check_qkv(desc, q, k, v, dout)
+    want = torch.float32 if desc.out_fp32 else torch.bfloat16
+    grads = [torch.empty(q.shape, dtype=want, device=q.device) for _ in range(3)]
+    n = ctypes.c_size_t(0)
+    _ok(lib().sparse_attn_bwd_scratch_size_heads(ctypes.byref(desc), _tiles_array(tiles),
+                                                 ctypes.byref(n)), "bwd_scratch_size_heads")
+    scratch = torch.empty(n.value, dtype=torch.uint8, device=q.device)
+    _ok(lib().sparse_attn_bwd_heads(ctypes.byref(desc), _tiles_array(tiles), _ptr(q), _ptr(k),
+                                    _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(workspace),
+                                    ctypes.c_size_t(workspace.numel()), _ptr(grads[0]),
+                                    _ptr(grads[1]), _ptr(grads[2]), _ptr(scratch),
+                                    ctypes.c_size_t(scratch.numel()), _stream(stream)),
+        "bwd_heads")
+    return tuple(grads)
+
+
+def block_heatmap_heads(desc: SaDesc, tiles, q, k, workspace, stream=None) -> torch.Tensor:
+    """The block max-pooled map [B*H, nb, nb] with per-head block shapes."""
+    _check_qkv(desc, q, k)
+    nb = desc.T * desc.Hh * desc.Ww // desc.N
+    heat = torch.empty((desc.B * desc.H, nb, nb), dtype=torch.float32, device=q.device)
+    n = ctypes.c_size_t(0)
+    _ok(lib().sparse_attn_block_heatmap_scratch_size_heads(
+        ctypes.byref(desc), _tiles_array(tiles), ctypes.byref(n)), "heatmap_scratch_size_heads")
+    scratch = torch.empty(n.value, dtype=torch.uint8, device=q.device)
+    _ok(lib().sparse_attn_block_heatmap_heads(ctypes.byref(desc), _tiles_array(tiles), _ptr(q),
+                                              _ptr(k), _ptr(workspace),
+                                              ctypes.c_size_t(workspace.numel()), _ptr(heat),
+                                              _ptr(scratch), ctypes.c_size_t(scratch.numel()),
+                                              _stream(stream)), "block_heatmap_heads")
+    return heat
 
 
 def heads_runs(desc: SaDesc, tiles):

@@ -131,6 +131,100 @@ sa_status sparse_attn_fwd_heads(const sa_desc* desc, const int* tiles, const voi
   });
 }
 
+sa_status sparse_attn_fwd_lse_heads(const sa_desc* desc, const int* tiles, const void* q,
+                                   const void* k, const void* v, const void* workspace,
+                                   size_t ws_bytes, void* out, float* lse, void* stream) {
+  size_t need = 0;
+  sa_status st = sparse_attn_workspace_size_heads(desc, tiles, &need);
+  if (st != SA_OK) return st;
+  if (workspace == nullptr || !aligned256(workspace)) return SA_ERR_INVALID_ARG;
+  if (ws_bytes < need) return SA_ERR_WORKSPACE;
+  if (lse == nullptr) return SA_ERR_INVALID_ARG;
+  const size_t hb = head_bytes(desc, 2);
+  const size_t ob = head_bytes(desc, desc->out_fp32 ? 4 : 2);
+  const size_t S = size_t(desc->T) * desc->Hh * desc->Ww;
+  return for_each_run(desc, tiles, nullptr, [&](const Run& r) {
+    return sparse_attn_fwd_lse(&r.sub, shift(q, hb * r.head0), shift(k, hb * r.head0),
+                               shift(v, hb * r.head0), shift(workspace, r.ws_off), r.ws_bytes,
+                               shift(out, ob * r.head0), lse + S * r.head0, stream);
+  });
+}
+
+// The runs execute one after another on the caller's stream, so one scratch
+// buffer of the largest run's size serves them all.
+sa_status sparse_attn_bwd_scratch_size_heads(const sa_desc* desc, const int* tiles,
+                                             size_t* bytes) {
+  if (bytes == nullptr) return SA_ERR_INVALID_ARG;
+  size_t most = 0;
+  const sa_status st = for_each_run(desc, tiles, nullptr, [&](const Run& r) {
+    size_t b = 0;
+    const sa_status s = sparse_attn_bwd_scratch_size(&r.sub, &b);
+    if (b > most) most = b;
+    return s;
+  });
+  if (st == SA_OK) *bytes = most;
+  return st;
+}
+
+sa_status sparse_attn_bwd_heads(const sa_desc* desc, const int* tiles, const void* q,
+                               const void* k, const void* v, const void* out, const void* dout,
+                               const float* lse, const void* workspace, size_t ws_bytes, void* dq,
+                               void* dk, void* dv, void* scratch, size_t scratch_bytes,
+                               void* stream) {
+  size_t need = 0, scr = 0;
+  sa_status st = sparse_attn_workspace_size_heads(desc, tiles, &need);
+  if (st != SA_OK) return st;
+  st = sparse_attn_bwd_scratch_size_heads(desc, tiles, &scr);
+  if (st != SA_OK) return st;
+  if (workspace == nullptr || !aligned256(workspace) || lse == nullptr) return SA_ERR_INVALID_ARG;
+  if (ws_bytes < need || scratch_bytes < scr) return SA_ERR_WORKSPACE;
+  const size_t hb = head_bytes(desc, 2);
+  const size_t ob = head_bytes(desc, desc->out_fp32 ? 4 : 2);
+  const size_t S = size_t(desc->T) * desc->Hh * desc->Ww;
+  return for_each_run(desc, tiles, nullptr, [&](const Run& r) {
+    return sparse_attn_bwd(&r.sub, shift(q, hb * r.head0), shift(k, hb * r.head0),
+                           shift(v, hb * r.head0), shift(out, ob * r.head0),
+                           shift(dout, hb * r.head0), lse + S * r.head0,
+                           shift(workspace, r.ws_off), r.ws_bytes, shift(dq, ob * r.head0),
+                           shift(dk, ob * r.head0), shift(dv, ob * r.head0), scratch,
+                           scratch_bytes, stream);
+  });
+}
+
+sa_status sparse_attn_block_heatmap_scratch_size_heads(const sa_desc* desc, const int* tiles,
+                                                       size_t* bytes) {
+  if (bytes == nullptr) return SA_ERR_INVALID_ARG;
+  size_t most = 0;
+  const sa_status st = for_each_run(desc, tiles, nullptr, [&](const Run& r) {
+    size_t b = 0;
+    const sa_status s = sparse_attn_block_heatmap_scratch_size(&r.sub, &b);
+    if (b > most) most = b;
+    return s;
+  });
+  if (st == SA_OK) *bytes = most;
+  return st;
+}
+
+sa_status sparse_attn_block_heatmap_heads(const sa_desc* desc, const int* tiles, const void* q,
+                                          const void* k, void* workspace, size_t ws_bytes,
+                                          float* heat, void* scratch, size_t scratch_bytes,
+                                          void* stream) {
+  size_t need = 0, scr = 0;
+  sa_status st = sparse_attn_workspace_size_heads(desc, tiles, &need);
+  if (st != SA_OK) return st;
+  st = sparse_attn_block_heatmap_scratch_size_heads(desc, tiles, &scr);
+  if (st != SA_OK) return st;
+  if (workspace == nullptr || !aligned256(workspace) || heat == nullptr) return SA_ERR_INVALID_ARG;
+  if (ws_bytes < need || scratch_bytes < scr) return SA_ERR_WORKSPACE;
+  const size_t hb = head_bytes(desc, 2);
+  const size_t nb = size_t(desc->T) * desc->Hh * desc->Ww / 64;  // the same for every shape
+  return for_each_run(desc, tiles, nullptr, [&](const Run& r) {
+    return sparse_attn_block_heatmap(&r.sub, shift(q, hb * r.head0), shift(k, hb * r.head0),
+                                     shift(workspace, r.ws_off), r.ws_bytes,
+                                     heat + nb * nb * r.head0, scratch, scratch_bytes, stream);
+  });
+}
+
 sa_status sparse_attn_check_heads(const sa_desc* desc, const int* tiles, const void* workspace,
                                   size_t ws_bytes, void* stream) {
   size_t need = 0;

@@ -221,6 +221,29 @@ sa_status sparse_attn_fwd_heads(const sa_desc* desc, const int* tiles, const voi
 sa_status sparse_attn_check_heads(const sa_desc* desc, const int* tiles, const void* workspace,
                                   size_t ws_bytes, void* stream);
 
+/* The forward with log-sum-exp, the gradients and the block max-pooled map
+ * with per-head shapes: the single-shape calls on every run's slices of the
+ * full [B, H, ...] tensors (lse [B*H][S], heat [B*H][nb][nb]) and of the
+ * workspace. The runs go one after another on `stream`, so one scratch
+ * buffer of the largest run's size (the *_scratch_size_heads calls) serves
+ * all of them. */
+sa_status sparse_attn_fwd_lse_heads(const sa_desc* desc, const int* tiles, const void* q,
+                                   const void* k, const void* v, const void* workspace,
+                                   size_t ws_bytes, void* out, float* lse, void* stream);
+sa_status sparse_attn_bwd_scratch_size_heads(const sa_desc* desc, const int* tiles,
+                                             size_t* bytes);
+sa_status sparse_attn_bwd_heads(const sa_desc* desc, const int* tiles, const void* q,
+                               const void* k, const void* v, const void* out, const void* dout,
+                               const float* lse, const void* workspace, size_t ws_bytes, void* dq,
+                               void* dk, void* dv, void* scratch, size_t scratch_bytes,
+                               void* stream);
+sa_status sparse_attn_block_heatmap_scratch_size_heads(const sa_desc* desc, const int* tiles,
+                                                       size_t* bytes);
+sa_status sparse_attn_block_heatmap_heads(const sa_desc* desc, const int* tiles, const void* q,
+                                          const void* k, void* workspace, size_t ws_bytes,
+                                          float* heat, void* scratch, size_t scratch_bytes,
+                                          void* stream);
+
 /* Host-only: run number `run` (0-based) as a single-shape problem: its
  * descriptor (*sub, B = 1, H = run length), first flattened head (*head0)
  * and workspace slice (*ws_offset, *ws_bytes), e.g. for sparse_attn_get_mask

@@ -186,3 +186,11 @@ def test_per_head_shapes_split_into_runs():
     n = ctypes.c_size_t()
     assert api.lib().sparse_attn_workspace_size_heads(ctypes.byref(d), None, ctypes.byref(n)) == \
         api.SA_ERR_INVALID_ARG
+    # one scratch buffer serves the runs of the gradient and map calls in turn:
+    # the largest run's size
+    arr = (ctypes.c_int * 36)(*[x for t in tiles for x in t])
+    for name, single in (("sparse_attn_bwd_scratch_size_heads", api.bwd_scratch_size),
+                         ("sparse_attn_block_heatmap_scratch_size_heads",
+                          api.heatmap_scratch_size)):
+        assert getattr(api.lib(), name)(ctypes.byref(d), arr, ctypes.byref(n)) == api.SA_OK
+        assert n.value == max(single(sub) for sub, *_ in runs)

@@ -135,3 +135,34 @@ def test_nabla_attention_methods_match_functional_calls():
     assert torch.equal(out, out2) and torch.equal(lse, lse2) and torch.equal(heat, heat2)
     for a, b in zip(grads, grads2):  # fp32 reductions in any order: equal to rounding
         assert torch.allclose(a, b, rtol=1e-5, atol=1e-6)
+
+
+def test_per_head_shapes_gradients_and_map_match_single_shape_runs():
+    w = W.W8K  # 12 heads
+    tiles = [(1, 8, 8)] * 4 + [(2, 4, 8)] * 4 + [(4, 4, 4)] * 2 + [(2, 4, 8)] * 2
+    desc = api.desc_for(w, out_fp32=True)
+    q, k, v = (to_dev(x) for x in W.make_inputs(w))
+    g = to_dev(W.make_output_grad(w))
+    ws = torch.empty(api.workspace_size_heads(desc, tiles), dtype=torch.uint8, device="cuda")
+    api.plan_heads(desc, tiles, q, k, ws)
+    out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device="cuda")
+    api.fwd_lse_heads(desc, tiles, q, k, v, ws, out, lse)
+    grads = api.bwd_heads(desc, tiles, q, k, v, out, g, lse, ws)
+    heat = api.block_heatmap_heads(desc, tiles, q, k, ws)
+    assert api.check_heads(desc, tiles, ws) == api.SA_OK
+    for sub, head0, _, _ in api.heads_runs(desc, tiles):
+        sl = slice(head0, head0 + sub.H)
+        qs, ks, vs, gs = (x[:, sl].contiguous() for x in (q, k, v, g))
+        ws1 = api.alloc_workspace(sub)
+        api.plan(sub, qs, ks, ws1)
+        o1 = torch.empty(qs.shape, dtype=torch.float32, device="cuda")
+        l1 = torch.empty(qs.shape[:3], dtype=torch.float32, device="cuda")
+        api.fwd_lse(sub, qs, ks, vs, ws1, o1, l1)
+        g1 = api.bwd(sub, qs, ks, vs, o1, gs, l1, ws1)
+        h1 = api.block_heatmap(sub, qs, ks, ws1)
+        assert api.check(sub, ws1) == api.SA_OK
+        assert torch.equal(out[:, sl], o1) and torch.equal(lse[:, sl], l1)
+        assert torch.equal(heat[sl], h1)
+        for a, b in zip(grads, g1):  # fp32 reductions in any order: equal to rounding
+            assert torch.allclose(a[:, sl], b, rtol=1e-5, atol=1e-6)
