@@ -11,11 +11,18 @@
  *                     + optional STA union  ->  block lists in a workspace;
  *   sparse_attn_fwd   exact attention over the kept (q-block, k-block) pairs,
  *                     written back in natural token order.
- * One plan may serve many fwd calls with the same Q/K statistics.
+ * One plan may serve many fwd calls with the same Q/K statistics. Around
+ * them: the gradients over the same mask (sparse_attn_fwd_lse,
+ * sparse_attn_bwd), the exact block max-pooled attention map that measures a
+ * mask's recall (sparse_attn_block_heatmap), per-head block shapes (*_heads),
+ * and the whole path as one CUDA graph launch (sparse_attn_graph_*).
  *
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller; the library
- *     allocates nothing and keeps no state between calls.
+ *     allocates nothing and keeps no state between calls, except the graph
+ *     object of sparse_attn_graph_create (owned by the caller until
+ *     sparse_attn_graph_destroy) and the built-in workspace of
+ *     sparse_attn_forward_noalloc.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *     stream). Argument errors are reported before anything is launched.
  *   - Q, K, V and the output use the natural video layout [B, H, S, d] with
