@@ -10,8 +10,12 @@ max |g - ref| <= REL_MAX * max |ref| and mean |g - ref| <= REL_MEAN * mean |ref|
 dQ and dK are the loosest: a row's dS sums to about zero (sum_j P (dP - D) = 0),
 so the bf16 rounding of its terms is large next to the sums they form. Seen on
 these cases: max 1.2e-2 (dQ), mean 6.0e-3 with bf16 outputs (their own
-rounding adds ~2^-10 on average) and 2.9e-3 with fp32 outputs; the bounds
-leave about a factor two.
+rounding adds ~2^-10 on average) and 2.9e-3 with fp32 outputs. The single-block
+case is the extreme: each row has only 64 keys, so with bf16 outputs the error
+D carries from the stored output (up to 2^-9 of |O|) meets the largest
+cancellation in dP - D: dQ mean 1.27e-2, against 2.0e-3 with fp32 outputs (and
+max errors of 1.0e-2 and 3.9e-3). The bounds leave a factor of about 1.6-2
+over what was seen.
 """
 import functools
 
@@ -27,7 +31,7 @@ pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
 
 REL_MAX = {False: 2.5e-2, True: 2.5e-2}    # keyed by out_fp32
-REL_MEAN = {False: 1.2e-2, True: 6e-3}
+REL_MEAN = {False: 2e-2, True: 6e-3}
 LSE_ABS = 1e-4
 
 CASES = [
@@ -35,6 +39,8 @@ CASES = [
     W.TINY.with_(name="odd_1x2x576x128", T=3, Hh=8, Ww=24, d=128),
     W.W8K_T248.with_(name="tile2x4x8_1x2x4096x128", T=8, Hh=16, Ww=32, H=2),
     W.W8K.with_(name="8k_1x2x8192x128_sta3", H=2),
+    # one block per head: a lone key tile with a one-entry list (a lone step)
+    W.TINY.with_(name="single_block_1x2x64x128", T=1, Hh=8, Ww=8, d=128),
 ]
 
 

@@ -31,6 +31,8 @@ CASES = [
     W.TINY.with_(name="odd_1x2x576x128", T=3, Hh=8, Ww=24, d=128),
     W.TINY.with_(name="odd_1x1x2880x64_sta", T=5, Hh=24, Ww=24, d=64, H=1, sta=(3, 3, 3)),
     W.W8K_T248.with_(name="tile2x4x8_1x2x4096x128", T=8, Hh=16, Ww=32, H=2),
+    # one block per head: a lone q-block in a lone tile, a lone k-block
+    W.TINY.with_(name="single_block_1x2x64x128", T=1, Hh=8, Ww=8, d=128),
     # 384 units of four q-blocks on at most 148 CTAs: several units per CTA
     W.TINY.with_(name="multi_1x48x2048x64", T=4, Hh=16, Ww=32, H=48),
 ]
