@@ -34,6 +34,7 @@ SYMBOLS = (
     "sparse_attn_graph_launch", "sparse_attn_graph_destroy", "sparse_attn_fwd_lse_heads",
     "sparse_attn_bwd_scratch_size_heads", "sparse_attn_bwd_heads",
     "sparse_attn_block_heatmap_scratch_size_heads", "sparse_attn_block_heatmap_heads",
+    "sparse_attn_plan_profile", "sparse_attn_plan_stage_name",
 )
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -88,10 +89,14 @@ def lib() -> ctypes.CDLL:
         L.sparse_attn_check_heads.argtypes = [dp, ip, vp, sz, vp]
         L.sparse_attn_heads_run.argtypes = [dp, ip, i32, dp, ip, ctypes.POINTER(sz),
                                             ctypes.POINTER(sz)]
+        L.sparse_attn_plan_profile.argtypes = [dp, vp, vp, vp, sz, i32,
+                                               ctypes.POINTER(ctypes.c_float), i32, ip, vp]
         L.sparse_attn_status_string.argtypes = [i32]
         L.sparse_attn_status_string.restype = ctypes.c_char_p
+        L.sparse_attn_plan_stage_name.argtypes = [i32]
+        L.sparse_attn_plan_stage_name.restype = ctypes.c_char_p
         for name in SYMBOLS:
-            if name != "sparse_attn_status_string":
+            if name not in ("sparse_attn_status_string", "sparse_attn_plan_stage_name"):
                 getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -157,6 +162,20 @@ def plan(desc: SaDesc, q: torch.Tensor, k: torch.Tensor, workspace: torch.Tensor
     _check_qkv(desc, q, k)
     _ok(lib().sparse_attn_plan(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(workspace),
                                workspace.numel(), _stream(stream)), "plan")
+
+
+def plan_profile(desc: SaDesc, q: torch.Tensor, k: torch.Tensor, workspace: torch.Tensor,
+                 reps: int = 5, stream=None) -> dict:
+    """Mean device time (µs) of each stage of the plan over ``reps`` plans
+    (blocks until they finish): {stage name: µs}."""
+    _check_qkv(desc, q, k)
+    cap = 16
+    us = (ctypes.c_float * cap)()
+    n = ctypes.c_int(0)
+    _ok(lib().sparse_attn_plan_profile(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(workspace),
+                                       workspace.numel(), int(reps), us, cap, ctypes.byref(n),
+                                       _stream(stream)), "plan_profile")
+    return {lib().sparse_attn_plan_stage_name(i).decode(): float(us[i]) for i in range(n.value)}
 
 
 def fwd(desc: SaDesc, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,

@@ -81,8 +81,14 @@ sa_status sparse_attn_workspace_size(const sa_desc* desc, size_t* bytes) {
   return SA_OK;
 }
 
-sa_status sparse_attn_plan(const sa_desc* desc, const void* q, const void* k, void* workspace,
-                           size_t ws_bytes, void* stream) {
+// Stages of the plan, in launch order (sparse_attn_plan_profile).
+const char* const kPlanStages[] = {"pool", "logits", "select", "union", "tile_order"};
+constexpr int kNumPlanStages = 5;
+
+// The plan; when ev is given (kNumPlanStages + 1 events) ev[0] is recorded
+// before the first launch and ev[i + 1] after stage i.
+static sa_status plan_impl(const sa_desc* desc, const void* q, const void* k, void* workspace,
+                           size_t ws_bytes, void* stream, cudaEvent_t* ev) {
   sa_status st = validate(desc);
   if (st != SA_OK) return st;
   if (q == nullptr || k == nullptr || !aligned(q, 16) || !aligned(k, 16))
@@ -93,11 +99,14 @@ sa_status sparse_attn_plan(const sa_desc* desc, const void* q, const void* k, vo
   const WsLayout w = make_ws_layout(g);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-  cudaError_t e = cudaMemsetAsync(at<uint32_t>(workspace, w.status), 0, 256, s);
+  cudaError_t e;
+  if (ev != nullptr && cudaEventRecord(ev[0], s) != cudaSuccess) return SA_ERR_CUDA;
+  e = cudaMemsetAsync(at<uint32_t>(workspace, w.status), 0, 256, s);
   if (e != cudaSuccess) return SA_ERR_CUDA;
   e = launch_pool(q, k, at<float>(workspace, w.qbar), at<float>(workspace, w.kbar),
                   at<float>(workspace, w.qsplit), at<float>(workspace, w.ksplit), g, s);
   if (e != cudaSuccess) return SA_ERR_CUDA;
+  if (ev != nullptr && cudaEventRecord(ev[1], s) != cudaSuccess) return SA_ERR_CUDA;
 
   MaskArgs m;
   std::memset(&m, 0, sizeof(m));
@@ -126,9 +135,49 @@ sa_status sparse_attn_plan(const sa_desc* desc, const void* q, const void* k, vo
   m.sta_h = sta ? desc->sta_h / 2 : -1;
   m.sta_w = sta ? desc->sta_w / 2 : -1;
   m.scale = (float)(1.0 / std::sqrt((double)g.d));
-  e = launch_mask(m, g, s);
+  e = launch_mask(m, g, s, ev != nullptr ? ev + 2 : nullptr);
   if (e != cudaSuccess) return SA_ERR_CUDA;
-  return cuda_status(launch_tile_order(m.tcnt, at<int32_t>(workspace, w.order), g, s));
+  if (ev != nullptr && cudaEventRecord(ev[4], s) != cudaSuccess) return SA_ERR_CUDA;
+  e = launch_tile_order(m.tcnt, at<int32_t>(workspace, w.order), g, s);
+  if (e != cudaSuccess) return SA_ERR_CUDA;
+  if (ev != nullptr && cudaEventRecord(ev[5], s) != cudaSuccess) return SA_ERR_CUDA;
+  return SA_OK;
+}
+
+sa_status sparse_attn_plan(const sa_desc* desc, const void* q, const void* k, void* workspace,
+                           size_t ws_bytes, void* stream) {
+  return plan_impl(desc, q, k, workspace, ws_bytes, stream, nullptr);
+}
+
+sa_status sparse_attn_plan_profile(const sa_desc* desc, const void* q, const void* k,
+                                   void* workspace, size_t ws_bytes, int reps, float* stage_us,
+                                   int max_stages, int* n_stages, void* stream) {
+  if (reps < 1 || stage_us == nullptr || n_stages == nullptr || max_stages < kNumPlanStages)
+    return SA_ERR_INVALID_ARG;
+  sa_status st = validate(desc);
+  if (st != SA_OK) return st;
+  *n_stages = kNumPlanStages;
+  for (int i = 0; i < kNumPlanStages; ++i) stage_us[i] = 0.f;
+  cudaEvent_t ev[kNumPlanStages + 1];
+  int made = 0;
+  for (; made <= kNumPlanStages; ++made)
+    if (cudaEventCreate(&ev[made]) != cudaSuccess) break;
+  st = made == kNumPlanStages + 1 ? SA_OK : SA_ERR_CUDA;
+  for (int r = 0; r < reps && st == SA_OK; ++r) {
+    st = plan_impl(desc, q, k, workspace, ws_bytes, stream, ev);
+    if (st == SA_OK && cudaEventSynchronize(ev[kNumPlanStages]) != cudaSuccess) st = SA_ERR_CUDA;
+    for (int i = 0; i < kNumPlanStages && st == SA_OK; ++i) {
+      float ms = 0.f;
+      if (cudaEventElapsedTime(&ms, ev[i], ev[i + 1]) != cudaSuccess) st = SA_ERR_CUDA;
+      stage_us[i] += ms * 1000.f / float(reps);
+    }
+  }
+  for (int i = 0; i < made; ++i) cudaEventDestroy(ev[i]);
+  return st;
+}
+
+const char* sparse_attn_plan_stage_name(int i) {
+  return (i >= 0 && i < kNumPlanStages) ? kPlanStages[i] : nullptr;
 }
 
 static sa_status fwd_impl(const sa_desc* desc, const void* q, const void* k, const void* v,

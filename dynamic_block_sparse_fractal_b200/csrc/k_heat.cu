@@ -1,6 +1,7 @@
 // Exact block max-pooled attention map (the reference target of the page
-// "Veda: Video Generation with Efficient Sparse Attention", section 2.1,
-// "Costruzione dell'Obiettivo"): for every (q-block, k-block) pair of a head,
+// "Veda - Diffusione Video Scalabile tramite Attenzione Sparsa Distillata",
+// gist.science/it/paper/2605.30325, section 2.1, "Costruzione
+// dell'Obiettivo"): for every (q-block, k-block) pair of a head,
 // the largest probability of the full, unmasked softmax attention inside the
 // N x N block. A quality signal for a block mask: how much of the real
 // attention its kept blocks carry.

@@ -544,11 +544,13 @@ cudaError_t launch_logits(const MaskArgs& a, const Geometry& g, int ld, cudaStre
 
 }  // namespace
 
-cudaError_t launch_mask(const MaskArgs& a, const Geometry& g, cudaStream_t stream) {
+cudaError_t launch_mask(const MaskArgs& a, const Geometry& g, cudaStream_t stream,
+                        cudaEvent_t* marks) {
   const int ld = logits_ld(g);
   cudaError_t e = g.d == 128 ? launch_logits<128>(a, g, ld, stream)
                              : launch_logits<64>(a, g, ld, stream);
   if (e != cudaSuccess) return e;
+  if (marks != nullptr && (e = cudaEventRecord(marks[0], stream)) != cudaSuccess) return e;
   const int vpl = (g.nb + 31) / 32;  // nb <= 3072 (checked by the entry points)
   if (vpl <= 4) e = launch_select<4>(a, g, ld, stream);
   else if (vpl <= 8) e = launch_select<8>(a, g, ld, stream);
@@ -557,6 +559,7 @@ cudaError_t launch_mask(const MaskArgs& a, const Geometry& g, cudaStream_t strea
   else if (vpl <= 64) e = launch_select<64>(a, g, ld, stream);
   else e = launch_select<96>(a, g, ld, stream);
   if (e != cudaSuccess) return e;
+  if (marks != nullptr && (e = cudaEventRecord(marks[1], stream)) != cudaSuccess) return e;
   const long items = long(g.BH) * g.ntile;
   const size_t warp_bytes = size_t(union_words_per_warp(g)) * sizeof(uint32_t);
   int wpc = int((48 * 1024) / warp_bytes);  // warps per CTA within 48 KB

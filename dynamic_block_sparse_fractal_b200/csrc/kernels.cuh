@@ -38,8 +38,10 @@ struct MaskArgs {
   int sta_t, sta_h, sta_w;  // half-widths (window / 2), -1 = no STA
   float scale;              // 1 / sqrt(d)
 };
-// Three launches: logits GEMM, row select, tile union.
-cudaError_t launch_mask(const MaskArgs& a, const Geometry& g, cudaStream_t stream);
+// Three launches: logits GEMM, row select, tile union. marks (optional, two
+// events) are recorded after the logits GEMM and after the row select.
+cudaError_t launch_mask(const MaskArgs& a, const Geometry& g, cudaStream_t stream,
+                        cudaEvent_t* marks = nullptr);
 
 // Per head: tiles sorted by descending union length (ties by tile index).
 cudaError_t launch_tile_order(const int32_t* tcnt, int32_t* order, const Geometry& g,

@@ -63,8 +63,8 @@ typedef struct sa_desc {
                         (1, P, P); otherwise a three-dimensional tile of pt
                         frames x ph rows x pw columns with pt*ph*pw == N, T % pt,
                         Hh % ph and Ww % pw all 0 (the head-aware tiling of
-                        "Veda: Video Generation with Efficient Sparse
-                        Attention", section 2.2); P is then not used. Block
+                        "Veda - Diffusione Video Scalabile tramite
+                        Attenzione Sparsa Distillata", section 2.2); P is then not used. Block
                         coordinates, tile pairing and the STA window are in
                         units of these tiles. */
 } sa_desc;
@@ -110,6 +110,21 @@ sa_status sparse_attn_workspace_size(const sa_desc* desc, size_t* bytes);
  * its previous contents are ignored and overwritten. */
 sa_status sparse_attn_plan(const sa_desc* desc, const void* q, const void* k,
                            void* workspace, size_t ws_bytes, void* stream);
+
+/* Diagnostics for measuring the plan's kernels. Runs sparse_attn_plan `reps`
+ * times on `stream` with CUDA events between its stages (the pages define no
+ * such split; it follows the steps listed above: pooling, reduced map, CDF
+ * threshold with the STA union, per-tile union lists, tile order), waits for
+ * each run, and writes every stage's mean device time in microseconds to
+ * stage_us[0 .. *n_stages - 1]. max_stages: the length of stage_us (at least
+ * the stage count, else SA_ERR_INVALID_ARG). Blocks the calling thread;
+ * creates and destroys its own events; not for stream capture.
+ * sparse_attn_plan_stage_name(i) names stage i (NULL outside the range). */
+sa_status sparse_attn_plan_profile(const sa_desc* desc, const void* q, const void* k,
+                                   void* workspace, size_t ws_bytes, int reps,
+                                   float* stage_us, int max_stages, int* n_stages,
+                                   void* stream);
+const char* sparse_attn_plan_stage_name(int i);
 
 /* O_i = sum over kept k-blocks of softmax(q_i . k_j / sqrt(d)) v_j for every
  * query token i, i.e. exact attention with every dropped N x N block at -inf
@@ -199,8 +214,9 @@ sa_status sparse_attn_forward_noalloc(const sa_desc* desc, const void* q,
                                       void* stream);
 
 /* ---- Per-head block shapes ------------------------------------------------
- * The head-aware tiling of "Veda: Video Generation with Efficient Sparse
- * Attention" (section 2.2, "Tiling Consapevole delle Teste"): each head may
+ * The head-aware tiling of "Veda - Diffusione Video Scalabile tramite
+ * Attenzione Sparsa Distillata" (gist.science/it/paper/2605.30325, section
+ * 2.2, "Tiling Consapevole delle Teste"): each head may
  * use its own block shape. tiles is a HOST array of B*H triples
  * (pt, ph, pw), in (batch, head) order; each must satisfy the single-shape
  * rules of sa_desc (pt*ph*pw == N, the grid divisible by it; 0,0,0 = the
@@ -317,8 +333,9 @@ sa_status sparse_attn_bwd(const sa_desc* desc, const void* q, const void* k, con
                           void* dv, void* scratch, size_t scratch_bytes, void* stream);
 
 /* ---- Block max-pooled attention map (mask diagnostics) -------------------
- * "Veda: Video Generation with Efficient Sparse Attention", section 2.1
- * ("Costruzione dell'Obiettivo"): the reference a block mask is measured
+ * "Veda - Diffusione Video Scalabile tramite Attenzione Sparsa Distillata"
+ * (gist.science/it/paper/2605.30325), section 2.1 ("Costruzione
+ * dell'Obiettivo"): the reference a block mask is measured
  * against is the full, unmasked attention P = softmax(Q K^T / sqrt(d)) of a
  * head, max-pooled over every N x N block:
  *   heat[bh][i][j] = max over q in block i, k in block j of P[q][k],

@@ -16,9 +16,10 @@ notes as well):
 
 * Fractal order: time outermost, then patch row, then patch column; inside a
   P x P patch the tokens are row-major (h % P, then w % P).
-* Three-dimensional tiles (the head-aware tiling of "Veda" on the page
-  "Veda: Video Generation with Efficient Sparse Attention", section 2.2,
-  "Tiling Consapevole delle Teste"): a tile shape (p_t, p_h, p_w) with
+* Three-dimensional tiles (the head-aware tiling of the page "Veda -
+  Diffusione Video Scalabile tramite Attenzione Sparsa Distillata"
+  (gist.science/it/paper/2605.30325), section 2.2, "Tiling Consapevole delle
+  Teste"): a tile shape (p_t, p_h, p_w) with
   p_t * p_h * p_w = N makes each block p_t consecutive frames of a
   p_h x p_w patch. Blocks are ordered (t // p_t, h // p_h, w // p_w) and the
   tokens inside a block (t % p_t, h % p_h, w % p_w), both row-major; the
@@ -253,11 +254,15 @@ def nabla_attention(q, k, v, T, Hh, Ww, P, N, thr, sta, mask=None):
 #   dV = P^T dO,  dP = dO V^T,  D_i = sum_c dO_ic O_ic = sum_j P_ij dP_ij,
 #   dS = P * (dP - D),  dQ = dS K / sqrt(d),  dK = dS^T Q / sqrt(d).
 
-def masked_attention_backward(qp, kp, vp, dop, mask, N):
+def masked_attention_backward(qp, kp, vp, dop, mask, N, o_stored=None):
     """Gradients of sum(O * dO) for O = masked_attention(qp, kp, vp, mask, N),
     and the rows' natural-log log-sum-exp of the kept scaled scores.
 
     qp, kp, vp, dop: [S, d] float64 (one head, fractal order); mask [nb, nb].
+    o_stored: optional [S, d] fractal-order output as a forward pass stored
+    it (for instance rounded to bf16). D_i then sums dO_i * o_stored_i
+    instead of dO_i * O_i, as a backward pass that reads its stored output
+    does; every other term is unchanged and exact.
     Returns (dq, dk, dv, lse): [S, d] x 3 and [S], fractal order.
     """
     S, d = qp.shape
@@ -274,7 +279,7 @@ def masked_attention_backward(qp, kp, vp, dop, mask, N):
         l = e.sum(axis=-1, keepdims=True)
         p = e / l
         lse[r] = (mx + np.log(l))[:, 0]
-        o = p @ vp[cols]
+        o = p @ vp[cols] if o_stored is None else np.asarray(o_stored, dtype=np.float64)[r]
         dp = dop[r] @ vp[cols].T
         D = (dop[r] * o).sum(axis=-1, keepdims=True)
         ds = p * (dp - D)
@@ -323,20 +328,23 @@ def masked_attention_backward_blocks(qp, kp, vp, dop, mask, N, qblocks, kblocks)
     return dq, dk, dv, lse
 
 
-def attention_backward_head(q, k, v, do, T, Hh, Ww, P, N, mask):
+def attention_backward_head(q, k, v, do, T, Hh, Ww, P, N, mask, o_stored=None):
     """One head in natural order: fractal flatten, masked_attention_backward,
-    inverse flatten. q, k, v, do: [S, d]. Returns (dq, dk, dv, lse) float64."""
+    inverse flatten. q, k, v, do (and o_stored, if given, a natural-order
+    [S, d] stored output): [S, d]. Returns (dq, dk, dv, lse) float64."""
     perm = fractal_order(T, Hh, Ww, P)
     qp, kp, vp, dop = (flatten(_as_f64(x), perm) for x in (q, k, v, do))
-    dq, dk, dv, lse = masked_attention_backward(qp, kp, vp, dop, mask, N)
+    os_p = None if o_stored is None else flatten(np.asarray(o_stored, dtype=np.float64), perm)
+    dq, dk, dv, lse = masked_attention_backward(qp, kp, vp, dop, mask, N, o_stored=os_p)
     lse_nat = np.empty_like(lse)
     lse_nat[perm] = lse
     return unflatten(dq, perm), unflatten(dk, perm), unflatten(dv, perm), lse_nat
 
 
 # --- Block max-pooled attention map (quality signal for a block mask) --------
-# The reference target of the page "Veda: Video Generation with Efficient
-# Sparse Attention", section 2.1 ("Costruzione dell'Obiettivo"): the full
+# The reference target of the page "Veda - Diffusione Video Scalabile tramite
+# Attenzione Sparsa Distillata" (gist.science/it/paper/2605.30325), section
+# 2.1 ("Costruzione dell'Obiettivo"): the full
 # attention matrix, max-pooled over the (query block, key block) regions.
 
 def block_heatmap(q, k, T, Hh, Ww, P, N):

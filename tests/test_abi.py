@@ -194,3 +194,24 @@ def test_per_head_shapes_split_into_runs():
                           api.heatmap_scratch_size)):
         assert getattr(api.lib(), name)(ctypes.byref(d), arr, ctypes.byref(n)) == api.SA_OK
         assert n.value == max(single(sub) for sub, *_ in runs)
+
+
+def test_plan_profile_names_and_rejection():
+    L = api.lib()
+    names = []
+    i = 0
+    while L.sparse_attn_plan_stage_name(i) is not None:
+        names.append(L.sparse_attn_plan_stage_name(i).decode())
+        i += 1
+    assert names and len(set(names)) == len(names)
+    assert L.sparse_attn_plan_stage_name(-1) is None
+    d = api.desc_for(W.TINY)
+    us = (ctypes.c_float * 16)()
+    n = ctypes.c_int(0)
+    need = api.workspace_size(d)
+    # too short an output array, zero repetitions: rejected before any launch
+    assert L.sparse_attn_plan_profile(ctypes.byref(d), FAKE, FAKE, FAKE, need, 1, us,
+                                      len(names) - 1, ctypes.byref(n), None) == \
+        api.SA_ERR_INVALID_ARG
+    assert L.sparse_attn_plan_profile(ctypes.byref(d), FAKE, FAKE, FAKE, need, 0, us, 16,
+                                      ctypes.byref(n), None) == api.SA_ERR_INVALID_ARG

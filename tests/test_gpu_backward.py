@@ -4,18 +4,23 @@ fp64 oracle, on the GPU's own mask, and the row log-sum-exp of the forward.
 Tolerances. The kernel recomputes P = 2^(s log2(e) - lse2) in fp32, rounds P
 and dS = P (dP - D) to bf16 for the tensor cores (relative 2^-9 each) and
 accumulates in fp32; D = rowsum(dO * O) uses the forward's output as stored
-(bf16 unless out_fp32), which moves D by up to 2^-9 of |O|. Errors are
-measured relative to the largest reference magnitude of each gradient:
-max |g - ref| <= REL_MAX * max |ref| and mean |g - ref| <= REL_MEAN * mean |ref|.
-dQ and dK are the loosest: a row's dS sums to about zero (sum_j P (dP - D) = 0),
-so the bf16 rounding of its terms is large next to the sums they form. Seen on
-these cases: max 1.2e-2 (dQ), mean 6.0e-3 with bf16 outputs (their own
-rounding adds ~2^-10 on average) and 2.9e-3 with fp32 outputs. The single-block
-case is the extreme: each row has only 64 keys, so with bf16 outputs the error
-D carries from the stored output (up to 2^-9 of |O|) meets the largest
-cancellation in dP - D: dQ mean 1.27e-2, against 2.0e-3 with fp32 outputs (and
-max errors of 1.0e-2 and 3.9e-3). The bounds leave a factor of about 1.6-2
-over what was seen.
+(bf16 unless out_fp32). Errors are measured relative to the largest reference
+magnitude of each gradient: max |g - ref| <= REL_MAX * max |ref| and
+mean |g - ref| <= REL_MEAN * mean |ref|. dQ and dK are the loosest: a row's dS
+sums to about zero (sum_j P (dP - D) = 0), so the bf16 rounding of its terms
+is large next to the sums they form. Seen on the multi-block cases: max
+1.2e-2 (dQ), mean 6.0e-3 with bf16 outputs and 2.9e-3 with fp32 outputs; the
+bounds leave a factor of about 2.
+
+The stored output. Rounding O to bf16 moves it by up to 2^-9 |O|, so D moves
+by up to 2^-9 sum_c |dO_c O_c|, and every dS_ij of the row by P_ij times that
+shift. With many kept keys per row dP - D is large next to the shift; with a
+single 64-key block per row (the one-block case) the row's 64 terms of dP - D
+cancel to within a few times the shift, which is where the bf16 case's dQ
+mean error of 1.27e-2 comes from (2.0e-3 with fp32 outputs). That case alone
+is held to SINGLE_BLOCK_REL_MEAN_BF16. The error source is also isolated:
+fed the GPU's own stored bf16 output for D (oracle o_stored), the oracle must
+agree with every bf16 case to the fp32-output bounds.
 """
 import functools
 
@@ -31,7 +36,8 @@ pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
 
 REL_MAX = {False: 2.5e-2, True: 2.5e-2}    # keyed by out_fp32
-REL_MEAN = {False: 2e-2, True: 6e-3}
+REL_MEAN = {False: 1.2e-2, True: 6e-3}
+SINGLE_BLOCK_REL_MEAN_BF16 = 2e-2          # one 64-key block per row, bf16 output
 LSE_ABS = 1e-4
 
 CASES = [
@@ -66,7 +72,8 @@ def gpu_grads(w, out_fp32):
     views = api.get_mask(desc, ws)
     mask = parity.lists_to_mask(views["cnt"].cpu().numpy(), views["idx"].cpu().numpy())
     host = lambda t: t.float().cpu().numpy().reshape(w.BH, w.S, w.d)
-    return (host(dq), host(dk), host(dv), lse.cpu().numpy().reshape(w.BH, w.S), mask)
+    return (host(dq), host(dk), host(dv), lse.cpu().numpy().reshape(w.BH, w.S), mask,
+            host(out))
 
 
 def rel_errors(got, ref):
@@ -74,10 +81,16 @@ def rel_errors(got, ref):
     return e.max() / np.abs(ref).max(), e.mean() / np.abs(ref).mean()
 
 
+def mean_bound(w, out_fp32):
+    if not out_fp32 and w.nb == 1:
+        return SINGLE_BLOCK_REL_MEAN_BF16
+    return REL_MEAN[out_fp32]
+
+
 @pytest.mark.parametrize("out_fp32", [False, True])
 @pytest.mark.parametrize("w", CASES, ids=[c.name for c in CASES])
 def test_backward_matches_oracle(w, out_fp32):
-    dq, dk, dv, lse, mask = gpu_grads(w, out_fp32)
+    dq, dk, dv, lse, mask, _ = gpu_grads(w, out_fp32)
     q, k, v = (x.reshape(w.BH, w.S, w.d) for x in W.make_inputs(w))
     g = W.make_output_grad(w).reshape(w.BH, w.S, w.d)
     for bh in range(w.BH):
@@ -88,7 +101,26 @@ def test_backward_matches_oracle(w, out_fp32):
             mx, mean = rel_errors(got, ref)
             print(f"{w.name} fp32={out_fp32} head {bh} {name}: max {mx:.2e} mean {mean:.2e}")
             assert mx <= REL_MAX[out_fp32], (name, bh, mx)
-            assert mean <= REL_MEAN[out_fp32], (name, bh, mean)
+            assert mean <= mean_bound(w, out_fp32), (name, bh, mean)
+
+
+@pytest.mark.parametrize("w", CASES, ids=[c.name for c in CASES])
+def test_backward_bf16_output_with_stored_D_meets_fp32_bounds(w):
+    # The same bf16-output gradients against the oracle whose D reads the
+    # GPU's stored bf16 output: with the one error source the bf16 output adds
+    # taken into the reference, the fp32-output bounds hold for every case.
+    dq, dk, dv, _, mask, out = gpu_grads(w, False)
+    q, k, v = (x.reshape(w.BH, w.S, w.d) for x in W.make_inputs(w))
+    g = W.make_output_grad(w).reshape(w.BH, w.S, w.d)
+    for bh in range(w.BH):
+        rq, rk, rv, _ = oracle.attention_backward_head(q[bh], k[bh], v[bh], g[bh], w.T, w.Hh,
+                                                       w.Ww, w.block, w.N, mask[bh],
+                                                       o_stored=out[bh])
+        for name, got, ref in (("dq", dq[bh], rq), ("dk", dk[bh], rk), ("dv", dv[bh], rv)):
+            mx, mean = rel_errors(got, ref)
+            print(f"{w.name} stored-O head {bh} {name}: max {mx:.2e} mean {mean:.2e}")
+            assert mx <= REL_MAX[True], (name, bh, mx)
+            assert mean <= REL_MEAN[True], (name, bh, mean)
 
 
 def test_backward_full_size_sampled_blocks():
@@ -96,7 +128,7 @@ def test_backward_full_size_sampled_blocks():
     # the benchmark: dQ and the log-sum-exp of three q-blocks and dK, dV of
     # three k-blocks per head, from the oracle's per-block form.
     w = W.HUNYUAN.with_(name="hunyuan_1x2x126720x128", H=2)
-    dq, dk, dv, lse, mask = gpu_grads(w, False)
+    dq, dk, dv, lse, mask, _ = gpu_grads(w, False)
     q, k, v = (x.reshape(w.BH, w.S, w.d) for x in W.make_inputs(w))
     g = W.make_output_grad(w).reshape(w.BH, w.S, w.d)
     perm = oracle.fractal_order(w.T, w.Hh, w.Ww, w.block)

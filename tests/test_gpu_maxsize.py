@@ -42,7 +42,7 @@ def test_max_blocks_heatmap_rows():
 
 def test_max_blocks_backward_sampled():
     w = W_MAX
-    dq, dk, dv, lse, mask = gpu_grads(w, False)
+    dq, dk, dv, lse, mask, _ = gpu_grads(w, False)
     q, k, v = (x.reshape(w.BH, w.S, w.d) for x in W.make_inputs(w))
     g = W.make_output_grad(w).reshape(w.BH, w.S, w.d)
     perm = oracle.fractal_order(w.T, w.Hh, w.Ww, w.block)

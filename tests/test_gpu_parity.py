@@ -55,9 +55,11 @@ def check_mask(w, gm, heads=None):
     M, Mn, A = oracle_mask(w, heads)
     sel = list(range(w.BH) if heads is None else heads)
     r = parity.compare_masks(gm[sel], M, Mn, A, w.thr)
+    print(f"{w.name} mask: {r}")
     assert r["bad"] == 0, r
     assert r["sta_missing"] == 0, r
     assert r["min_mass_margin"] >= -parity.MASK_BAND, r
+    assert r["band_flips"] <= parity.max_band_flips(len(sel) * w.nb), r
     return r
 
 
@@ -79,6 +81,37 @@ def check_out_sampled(w, out, gm, heads, n_tok=96, seed=0, bf16_out=True):
                                           tokens=toks))
         got.append(out[bh][toks])
     r = parity.out_check(np.concatenate(got), np.concatenate(refs), bf16_out)
+    assert r["ok"], r
+    return r
+
+
+def check_out_qblocks(w, out, gm, views, desc, heads, per_head=32, seed=0, bf16_out=True):
+    """Whole q-blocks (all N rows) of every head in ``heads`` against the
+    oracle on the GPU's mask: per head the two q-blocks of each of the four
+    tiles with the longest union lists, of the two tiles with the shortest,
+    and of random other tiles up to ``per_head`` q-blocks."""
+    q, k, v = host_inputs(w)
+    perm = oracle.fractal_order(w.T, w.Hh, w.Ww, w.block)
+    tcnt = views["tile_cnt"].cpu().numpy()
+    rng = np.random.default_rng(seed)
+    N, worst = w.N, None
+    got, refs = [], []
+    for bh in heads:
+        order = np.argsort(-tcnt[bh], kind="stable")
+        tiles = list(order[:4]) + list(order[-2:])
+        rest = [t for t in rng.permutation(order.size) if t not in tiles]
+        blocks = []
+        for t in tiles + rest:
+            qa, qb = api.tile_blocks(desc, int(t))
+            blocks += [qa] + ([qb] if qb >= 0 else [])
+            if len(blocks) >= per_head:
+                break
+        rows = np.concatenate([np.arange(b * N, (b + 1) * N) for b in blocks])
+        qp, kp, vp = (oracle.flatten(oracle.widen_bf16(x[bh]), perm) for x in (q, k, v))
+        refs.append(oracle.masked_attention(qp, kp, vp, gm[bh], N, rows=rows))
+        got.append(out[bh][perm[rows]])
+    r = parity.out_check(np.concatenate(got), np.concatenate(refs), bf16_out)
+    print(f"{w.name} whole q-blocks ({per_head} per head, {len(heads)} heads): {r}")
     assert r["ok"], r
     return r
 
@@ -264,6 +297,46 @@ def test_deterministic_and_plan_reuse():
     assert api.check(desc, ws1) == api.SA_OK
 
 
+@pytest.mark.parametrize("step", ["drift", "next_seed"])
+def test_stale_plan_on_next_step_inputs_matches_oracle(step):
+    # Plan reuse across denoising steps (the SVG2 page's centroid cache, its
+    # section C.1; the TRA page's "Riutilizzo Cross-Step"; the Veda page's
+    # temporal caching of tile scores): the mask planned on step t's Q, K
+    # serves the forward of step t+1. The result must be the oracle's exact
+    # attention on step t+1's tensors under step t's mask, both through a
+    # direct call and through a forward-only graph replay.
+    w = W.W8K
+    q, k, v = host_inputs(w)
+    if step == "drift":
+        q2, k2, v2 = W.drift_inputs(w, (q, k, v), eps=0.05)
+    else:
+        q2, k2, v2 = (x.reshape(w.BH, w.S, w.d)
+                      for x in W.make_inputs(w.with_(seed=w.seed + 1)))
+    desc = api.desc_for(w)
+    ws = api.alloc_workspace(desc)
+    api.plan(desc, to_dev(q, w), to_dev(k, w), ws)
+    views = api.get_mask(desc, ws)
+    stale = parity.lists_to_mask(views["cnt"].cpu().numpy(), views["idx"].cpu().numpy())
+    check_mask(w, stale)  # step t's mask is the oracle's for step t's tensors
+    qd, kd, vd = to_dev(q2, w), to_dev(k2, w), to_dev(v2, w)
+    out = torch.empty_like(qd)
+    api.fwd(desc, qd, kd, vd, ws, out)
+    out_g = torch.empty_like(qd)
+    graph = api.AttentionGraph(desc, qd, kd, vd, ws, out_g, with_plan=False)
+    graph.launch()
+    torch.cuda.synchronize()
+    graph.close()
+    assert api.check(desc, ws) == api.SA_OK
+    ref, _ = oracle.nabla_attention(q2, k2, v2, w.T, w.Hh, w.Ww, w.block, w.N, w.thr, w.sta,
+                                    mask=stale)
+    for o in (out, out_g):
+        r = parity.out_check(o.float().cpu().numpy().reshape(w.BH, w.S, w.d), ref, True)
+        assert r["ok"], r
+    M2, _, _ = oracle.nabla_mask(q2, k2, w.T, w.Hh, w.Ww, w.block, w.N, w.thr, w.sta)
+    print(f"{step}: blocks whose keep decision changed between the steps: "
+          f"{int((M2 != stale).sum())} of {stale.size}")
+
+
 def test_device_timeout_is_reported_and_context_survives():
     w = W.TINY
     q, k, v = (to_dev(x, w) for x in host_inputs(w))
@@ -289,10 +362,10 @@ def test_wan_full_size():
 
 def test_hunyuan_full_size():
     w = W.HUNYUAN
-    out, gm, *_ = run(w)
+    out, gm, views, desc, _ = run(w)
     r = check_mask(w, gm)
-    assert r["density"] < 0.2, r
-    check_out_sampled(w, out, gm, heads=(0, 13, 23), n_tok=64)
+    assert r["density"] <= 0.1, r  # the workload's 90% block sparsity
+    check_out_qblocks(w, out, gm, views, desc, heads=range(w.BH), per_head=32)
 
 
 SWEEP_FULL = [0, 7, 14, 21, 28, 35, 47]  # spans thr, STA on/off and every scale

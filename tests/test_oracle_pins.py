@@ -9,6 +9,7 @@ confirm that some pin catches each of them.
 import itertools
 import math
 import os
+from fractions import Fraction
 
 import numpy as np
 import pytest
@@ -522,7 +523,7 @@ _orig_masked = nabla.masked_attention
 _orig_bwd = nabla.masked_attention_backward
 
 
-def _mut_backward_no_D(qp, kp, vp, dop, mask, N):
+def _mut_backward_no_D(qp, kp, vp, dop, mask, N, o_stored=None):
     # dS = P * dP (the -D term dropped): only dQ and dK change
     S, d = qp.shape
     o = _orig_masked(qp, kp, vp, mask, N)
@@ -541,9 +542,36 @@ def _mut_backward_no_D(qp, kp, vp, dop, mask, N):
     return dq, dk, dv, lse
 
 
-def _mut_backward_dk_unscaled(qp, kp, vp, dop, mask, N):
+def _mut_backward_dk_unscaled(qp, kp, vp, dop, mask, N, o_stored=None):
     dq, dk, dv, lse = _orig_bwd(qp, kp, vp, dop, mask, N)
     return dq, dk * np.sqrt(qp.shape[-1]), dv, lse
+
+
+def golden_recall(golden_dir):
+    out = []
+    for ln in _rows(os.path.join(golden_dir, "heat_recall.txt")):
+        h, m, r = (x.strip() for x in ln.split("|"))
+        H = np.array([[float(x) for x in row.split()] for row in h.split(";")])
+        M = np.array([[int(x) for x in row.split()] for row in m.split(";")], dtype=bool)
+        out.append((H, M, float(Fraction(r))))
+    return out
+
+
+def pin_recall_golden(golden_dir):
+    for H, M, expect in golden_recall(golden_dir):
+        got = oracle.heat_recall(H, M)
+        assert abs(got - expect) < 1e-12, (got, expect)
+
+
+def _mut_recall_pooled(H, M):
+    H = np.asarray(H, dtype=np.float64)
+    return float((H * M).sum() / H.sum())
+
+
+def _mut_recall_over_columns(H, M):
+    H = np.asarray(H, dtype=np.float64)
+    return float(np.mean((H * M).sum(axis=0) / H.sum(axis=0)))
+
 
 MUTANTS = [
     ("fractal_order", _mut_fractal_inner_transposed, "fractal"),
@@ -560,6 +588,8 @@ MUTANTS = [
     ("masked_attention", _mut_attention_no_scale, "attention"),
     ("masked_attention_backward", _mut_backward_no_D, "backward"),
     ("masked_attention_backward", _mut_backward_dk_unscaled, "backward"),
+    ("heat_recall", _mut_recall_pooled, "recall"),
+    ("heat_recall", _mut_recall_over_columns, "recall"),
 ]
 
 
@@ -608,6 +638,7 @@ def test_planted_mistake_is_caught(name, mutant, area, golden_dir, monkeypatch):
         "sta": [lambda: pin_sta_golden(golden_dir)],
         "attention": [pin_attention_own_patch, pin_attention_dense_is_sdpa],
         "backward": [pin_backward_finite_differences, pin_backward_dense_is_torch_autograd],
+        "recall": [lambda: pin_recall_golden(golden_dir)],
     }[area]
     caught = 0
     for pin in pins:
@@ -663,3 +694,33 @@ def test_block_heatmap_closed_forms_and_bounds():
     assert oracle.heat_recall(H, ~M) == 1.0 and oracle.heat_recall(H, M) == 0.0
     top = H >= np.sort(H, axis=1)[:, -2:-1]  # two largest per row
     assert 0.0 < oracle.heat_recall(H, top) < 1.0
+
+
+def test_heat_recall_golden(golden_dir):
+    pin_recall_golden(golden_dir)
+
+
+def test_backward_stored_output_shifts_only_the_D_term():
+    # D_i = sum_c dO_ic o_ic enters only through dS = P (dP - D). Replacing
+    # the exact O by a stored copy moves D by delta_i = sum_c dO_ic
+    # (stored - exact)_ic and therefore dQ_i by -delta_i / sqrt(d) times
+    # sum_j P_ij k_j, which is the forward attention with K in place of V.
+    rng = np.random.default_rng(61)
+    S, d, N = 256, 8, 64
+    nb = S // N
+    qp, kp, vp, dop = (rng.standard_normal((S, d)) for _ in range(4))
+    mask = rng.random((nb, nb)) < 0.5
+    mask[np.arange(nb), np.arange(nb)] = True
+    o = oracle.masked_attention(qp, kp, vp, mask, N)
+    exact = oracle.masked_attention_backward(qp, kp, vp, dop, mask, N)
+    same = oracle.masked_attention_backward(qp, kp, vp, dop, mask, N, o_stored=o)
+    for a, b in zip(exact, same):
+        assert np.abs(a - b).max() < 1e-12
+    stored = o + 1e-3 * rng.standard_normal(o.shape)
+    moved = oracle.masked_attention_backward(qp, kp, vp, dop, mask, N, o_stored=stored)
+    delta = (dop * (stored - o)).sum(axis=-1)
+    pk = oracle.masked_attention(qp, kp, kp, mask, N)
+    expect_dq = exact[0] - delta[:, None] * pk / np.sqrt(d)
+    assert np.abs(moved[0] - expect_dq).max() < 1e-12
+    assert np.abs(moved[2] - exact[2]).max() < 1e-12 and np.abs(moved[3] - exact[3]).max() < 1e-12
+    assert np.abs(moved[0] - exact[0]).max() > 1e-6  # the substitution is live

@@ -32,3 +32,15 @@ def test_sweep_variants():
     assert len(names) == W.N_SWEEP == 48
     w = W.sweep(0)
     assert w.thr == 0.0 and w.sta == (0, 0, 0) and w.scale == 0.0
+
+
+def test_drift_inputs_is_a_small_seeded_bf16_step():
+    w = W.TINY
+    q, k, v = W.make_inputs(w)
+    a = W.drift_inputs(w, (q, k, v), eps=0.05)
+    b = W.drift_inputs(w, (q, k, v), eps=0.05)
+    for x, y, z in zip((q, k, v), a, b):
+        assert y.dtype == np.uint16 and y.shape == x.shape and np.array_equal(y, z)
+        dx = W.bf16_bits_to_f32(y) - W.bf16_bits_to_f32(x)
+        assert 0.03 < float(np.std(dx)) < 0.07  # eps, plus bf16 rounding of the sum
+        assert not np.array_equal(x, y)
