@@ -1,4 +1,5 @@
-"""CPU fp64 oracle for NABLA block-sparse video attention.
+"""CPU fp64 oracle for NABLA block-sparse video attention (nabla.py) and for
+the Token Radius Attention block mask (tra.py).
 
 TEST INFRASTRUCTURE ONLY: the reference the CUDA path is checked against.
 Only the tests, the smoke check and the benchmark's CPU-baseline leg may
@@ -9,4 +10,7 @@ from .nabla import (  # noqa: F401
     block_coords, sta_keep, pooled_head, nabla_mask, masked_attention,
     attention_head, nabla_attention, tile_shape, block_heatmap, block_heatmap_rows, heat_recall,
     masked_attention_backward, masked_attention_backward_blocks, attention_backward_head,
+)
+from .tra import (  # noqa: F401
+    token_entropy, entropy_budget, budget_radius2, radius_support, radius_block_mask, tra_mask,
 )
