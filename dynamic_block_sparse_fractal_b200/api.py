@@ -35,6 +35,7 @@ SYMBOLS = (
     "sparse_attn_bwd_scratch_size_heads", "sparse_attn_bwd_heads",
     "sparse_attn_block_heatmap_scratch_size_heads", "sparse_attn_block_heatmap_heads",
     "sparse_attn_plan_profile", "sparse_attn_plan_stage_name",
+    "sparse_attn_token_entropy", "sparse_attn_plan_radius",
 )
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -46,6 +47,10 @@ class SaDesc(ctypes.Structure):
                 ("sta_t", ctypes.c_int), ("sta_h", ctypes.c_int), ("sta_w", ctypes.c_int),
                 ("out_fp32", ctypes.c_int), ("debug_flags", ctypes.c_int),
                 ("pt", ctypes.c_int), ("ph", ctypes.c_int), ("pw", ctypes.c_int)]
+
+
+class SaRadius(ctypes.Structure):
+    _fields_ = [("tau", ctypes.c_float), ("gamma", ctypes.c_float), ("vote_min", ctypes.c_int)]
 
 
 class SaMaskViews(ctypes.Structure):
@@ -91,6 +96,8 @@ def lib() -> ctypes.CDLL:
                                             ctypes.POINTER(sz)]
         L.sparse_attn_plan_profile.argtypes = [dp, vp, vp, vp, sz, i32,
                                                ctypes.POINTER(ctypes.c_float), i32, ip, vp]
+        L.sparse_attn_token_entropy.argtypes = [dp, vp, vp, vp, sz, vp, vp]
+        L.sparse_attn_plan_radius.argtypes = [dp, ctypes.POINTER(SaRadius), vp, vp, sz, vp]
         L.sparse_attn_status_string.argtypes = [i32]
         L.sparse_attn_status_string.restype = ctypes.c_char_p
         L.sparse_attn_plan_stage_name.argtypes = [i32]
@@ -162,6 +169,34 @@ def plan(desc: SaDesc, q: torch.Tensor, k: torch.Tensor, workspace: torch.Tensor
     _check_qkv(desc, q, k)
     _ok(lib().sparse_attn_plan(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(workspace),
                                workspace.numel(), _stream(stream)), "plan")
+
+
+def token_entropy(desc: SaDesc, q: torch.Tensor, k: torch.Tensor, workspace: torch.Tensor,
+                  entropy: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Entropy (nats) of every query's full attention row: fp32 [B, H, S]."""
+    _check_qkv(desc, q, k)
+    if entropy is None:
+        entropy = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    if entropy.dtype != torch.float32 or entropy.shape != q.shape[:3] or \
+            not entropy.is_contiguous():
+        raise ValueError("entropy must be a contiguous float32 tensor shaped [B, H, S]")
+    _ok(lib().sparse_attn_token_entropy(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(workspace),
+                                        workspace.numel(), _ptr(entropy), _stream(stream)),
+        "token_entropy")
+    return entropy
+
+
+def plan_radius(desc: SaDesc, tau: float, gamma: float, vote_min: int, entropy: torch.Tensor,
+                workspace: torch.Tensor, stream=None) -> None:
+    """Token Radius Attention block mask from per-token entropies (fp32
+    [B, H, S], natural order) into ``workspace``, in sparse_attn_plan's format."""
+    if entropy.dtype != torch.float32 or not entropy.is_contiguous() or \
+            entropy.numel() != desc.B * desc.H * desc.T * desc.Hh * desc.Ww:
+        raise ValueError("entropy must be a contiguous float32 tensor shaped [B, H, S]")
+    r = SaRadius(float(tau), float(gamma), int(vote_min))
+    _ok(lib().sparse_attn_plan_radius(ctypes.byref(desc), ctypes.byref(r), _ptr(entropy),
+                                      _ptr(workspace), workspace.numel(), _stream(stream)),
+        "plan_radius")
 
 
 def plan_profile(desc: SaDesc, q: torch.Tensor, k: torch.Tensor, workspace: torch.Tensor,

@@ -318,6 +318,71 @@ sa_status sparse_attn_block_heatmap(const sa_desc* desc, const void* q, const vo
   return cuda_status(launch_heat(a, g, s));
 }
 
+sa_status sparse_attn_token_entropy(const sa_desc* desc, const void* q, const void* k,
+                                    void* workspace, size_t ws_bytes, float* entropy,
+                                    void* stream) {
+  sa_status st = validate(desc);
+  if (st != SA_OK) return st;
+  if (q == nullptr || k == nullptr || entropy == nullptr || !aligned(q, 16) || !aligned(k, 16) ||
+      !aligned(entropy, 4))
+    return SA_ERR_INVALID_ARG;
+  const Geometry g = make_geometry(*desc);
+  st = check_ws(g, workspace, ws_bytes);
+  if (st != SA_OK) return st;
+  const WsLayout w = make_ws_layout(g);
+  HeatArgs a;
+  std::memset(&a, 0, sizeof(a));
+  if (!encode_tile_map(&a.map_q, q, g.BH, g.T, g.Hh, g.Ww, g.d, g.pt, g.ph, g.pw) ||
+      !encode_tile_map(&a.map_k, k, g.BH, g.T, g.Hh, g.Ww, g.d, g.pt, g.ph, g.pw))
+    return SA_ERR_CUDA;
+  a.entropy = entropy;
+  a.status = at<uint32_t>(workspace, w.status);
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)g.d));
+  a.debug_flags = desc->debug_flags;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(a.status, 0, sizeof(uint32_t), s) != cudaSuccess) return SA_ERR_CUDA;
+  return cuda_status(launch_heat(a, g, s));
+}
+
+sa_status sparse_attn_plan_radius(const sa_desc* desc, const sa_radius* radius,
+                                  const float* entropy, void* workspace, size_t ws_bytes,
+                                  void* stream) {
+  sa_status st = validate(desc);
+  if (st != SA_OK) return st;
+  if (radius == nullptr || entropy == nullptr || !aligned(entropy, 4)) return SA_ERR_INVALID_ARG;
+  if (!(radius->tau > 0.0f && std::isfinite(radius->tau)) ||
+      !(radius->gamma >= 0.0f && std::isfinite(radius->gamma)) || radius->vote_min < 1 ||
+      radius->vote_min > desc->N)
+    return SA_ERR_INVALID_ARG;
+  const Geometry g = make_geometry(*desc);
+  if (!radius_supported(g)) return SA_ERR_UNSUPPORTED;
+  st = check_ws(g, workspace, ws_bytes);
+  if (st != SA_OK) return st;
+  const WsLayout w = make_ws_layout(g);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(at<uint32_t>(workspace, w.status), 0, 256, s) != cudaSuccess)
+    return SA_ERR_CUDA;
+  RadiusArgs r;
+  r.entropy = entropy;
+  r.bits = at<uint32_t>(workspace, w.bits);
+  r.cnt = at<int32_t>(workspace, w.cnt);
+  r.idx = at<int32_t>(workspace, w.idx);
+  r.tau = radius->tau;
+  r.gamma = radius->gamma;
+  r.vote_min = radius->vote_min;
+  if (launch_radius(r, g, s) != cudaSuccess) return SA_ERR_CUDA;
+  MaskArgs m;
+  std::memset(&m, 0, sizeof(m));
+  m.bits = r.bits;
+  m.cnt = r.cnt;
+  m.idx = r.idx;
+  m.tcnt = at<int32_t>(workspace, w.tcnt);
+  m.tidx = at<int32_t>(workspace, w.tidx);
+  m.status = at<uint32_t>(workspace, w.status);
+  if (launch_union(m, g, s) != cudaSuccess) return SA_ERR_CUDA;
+  return cuda_status(launch_tile_order(m.tcnt, at<int32_t>(workspace, w.order), g, s));
+}
+
 sa_status sparse_attn_permute(const sa_desc* desc, const void* x, void* y, int inverse,
                               void* stream) {
   const sa_status st = validate(desc);

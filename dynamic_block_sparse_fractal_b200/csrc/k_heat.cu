@@ -52,15 +52,20 @@ struct __align__(1024) HeatSmem {
   uint64_t lse_bar[2];                  // [tile]: both halves' (max, sum) written
   uint64_t drain;
   float2 ml[2][2][2][128];              // [unit parity][tile][half][row]: (max, sum)
+  float xs[2][2][2][128];               // the same: sum of 2^(x - max) (x - max)
   uint32_t tmem_base;
   int abort;
 };
 
 // Sum over the 64 columns of 2^(s * sl2 - m), two columns per packed op;
-// kHeatPolyPairsPer8 of every 8 pairs take the FMA-pipe exp2.
-__device__ __forceinline__ float exp2_row_sum(const uint32_t (&sv)[64], uint64_t sl2x2, float m) {
+// kHeatPolyPairsPer8 of every 8 pairs take the FMA-pipe exp2. With ENT, also
+// the sum of 2^(x - m) * (x - m) (x = s * sl2), for the row's entropy.
+template <bool ENT>
+__device__ __forceinline__ float exp2_row_sum(const uint32_t (&sv)[64], uint64_t sl2x2, float m,
+                                              float& xsum) {
   const uint64_t negm2 = f2_pack(-m, -m);
   uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};
+  uint64_t xs2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
     const uint64_t x2 = f2_fma(
@@ -73,8 +78,13 @@ __device__ __forceinline__ float exp2_row_sum(const uint32_t (&sv)[64], uint64_t
     else
       e2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
     rs2[i & 3] = f2_add(rs2[i & 3], e2);
+    if (ENT) xs2[i & 3] = f2_fma(e2, x2, xs2[i & 3]);
   }
   float lo, hi;
+  if (ENT) {
+    f2_unpack(f2_add(f2_add(xs2[0], xs2[1]), f2_add(xs2[2], xs2[3])), lo, hi);
+    xsum = lo + hi;
+  }
   f2_unpack(f2_add(f2_add(rs2[0], rs2[1]), f2_add(rs2[2], rs2[3])), lo, hi);
   return lo + hi;
 }
@@ -94,7 +104,9 @@ __device__ __forceinline__ void heat_unit(const Geometry& g, long u, int& bh, in
 
 }  // namespace
 
-template <int D>
+// MAP: write the block max-pooled map (scratch + reduction); ENT: write each
+// query row's entropy. At least one of the two.
+template <int D, bool MAP, bool ENT>
 __global__ void __launch_bounds__(kHThreads, 1)
     heat_kernel(const __grid_constant__ HeatArgs a, const Geometry g) {
   extern __shared__ uint8_t h_raw[];
@@ -242,7 +254,7 @@ __global__ void __launch_bounds__(kHThreads, 1)
     const uint32_t t_lane =
         tmem + (uint32_t(quad * 32) << 16) + uint32_t(x) * 256u + uint32_t(e) * 64u;
     // this thread's scratch column: entry b at mine[b * kHRows]
-    float* mine = a.scratch + size_t(blockIdx.x) * kHRows * g.nb + x * 128 + r;
+    float* mine = MAP ? a.scratch + size_t(blockIdx.x) * kHRows * g.nb + x * 128 + r : nullptr;
     const float sl2 = a.scale_log2;
     const uint64_t sl2x2 = f2_pack(sl2, sl2);
     bool ok = true;
@@ -250,7 +262,10 @@ __global__ void __launch_bounds__(kHThreads, 1)
     for (long u = blockIdx.x; ok && u < units; u += gridDim.x, ++it) {
       int bh, base;
       heat_unit(g, u, bh, base);
-      float m = -INFINITY, l = 0.f;  // log2-domain running max and sum over this half
+      // log2-domain running max and sum over this half; xs = sum of
+      // 2^(x - m) (x - m) for the entropy (relative to m, so that no large
+      // values cancel)
+      float m = -INFINITY, l = 0.f, xs = 0.f;
       for (int j = 0; j < nsteps; ++j, ++op) {
         const int buf = op & 1;
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sm.s_full[x][buf], (op >> 1) & 1, abort));
@@ -274,16 +289,21 @@ __global__ void __launch_bounds__(kHThreads, 1)
           mq[(i >> 1) & 3] =
               max3(mq[(i >> 1) & 3], __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
         const float bmax = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
-        mine[size_t(2 * j + e) * kHRows] = bmax;
+        if (MAP) mine[size_t(2 * j + e) * kHRows] = bmax;
         const float m_new = fmaxf(m, bmax * sl2);
-        l *= ex2_approx(m - m_new);  // m = -inf at first: 2^-inf = 0
+        const float alpha = ex2_approx(m - m_new);  // m = -inf at first: 2^-inf = 0
+        if (ENT) xs = l > 0.f ? alpha * fmaf(l, m - m_new, xs) : 0.f;
+        l *= alpha;
         m = m_new;
-        l += exp2_row_sum(sv, sl2x2, m);
+        float xsj = 0.f;
+        l += exp2_row_sum<ENT>(sv, sl2x2, m, xsj);
+        if (ENT) xs += xsj;
       }
       if (!ok) break;
       // ---- the row's two halves meet: lse2 over all keys (both threads of
       // the row compute the same value)
       sm.ml[it & 1][x][e][r] = make_float2(m, l);
+      if (ENT) sm.xs[it & 1][x][e][r] = xs;
       mbar_arrive(&sm.lse_bar[x]);
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sm.lse_bar[x], it & 1, abort));
       if (!ok) break;
@@ -292,9 +312,20 @@ __global__ void __launch_bounds__(kHThreads, 1)
       const float ll = (e == 0 ? l * ex2_approx(m - mm) + o.y * ex2_approx(o.x - mm)
                                : o.y * ex2_approx(o.x - mm) + l * ex2_approx(m - mm));
       const float lse2 = mm + __log2f(ll);
-      // ---- this unit's map rows, blocks 2i + e
       const int qblk = base + 2 * x + half;  // uniform across the warp
       if (qblk >= g.nb) continue;
+      if (ENT && e == 0) {
+        // H = -sum p ln p with p = 2^(x - lse2): ln 2 (log2 L - XS / L), L and
+        // XS the row's sums relative to mm (the halves rescaled, XS shifted)
+        const float ox = sm.xs[it & 1][x][1][r];
+        const float a0 = ex2_approx(m - mm), a1 = ex2_approx(o.x - mm);
+        const float X0 = l > 0.f ? a0 * fmaf(l, m - mm, xs) : 0.f;
+        const float X1 = o.y > 0.f ? a1 * fmaf(o.y, o.x - mm, ox) : 0.f;
+        const float H = 0.6931471805599453f * (__log2f(ll) - (X0 + X1) / ll);
+        a.entropy[size_t(bh) * g.S + block_row_token(g, qblk, r & 63)] = H;
+      }
+      if (!MAP) continue;
+      // ---- this unit's map rows, blocks 2i + e
       int* out = reinterpret_cast<int*>(a.heat) + (size_t(bh) * g.nb + qblk) * g.nb + e;
       const int nbe = (g.nb - e + 1) / 2;  // blocks of this parity
       for (int b0 = 0; b0 < nbe; b0 += 32) {
@@ -327,17 +358,29 @@ __global__ void __launch_bounds__(kHThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-template <int D>
-static cudaError_t launch_heat_d(const HeatArgs& a, const Geometry& g, cudaStream_t stream) {
+template <int D, bool MAP, bool ENT>
+static cudaError_t launch_heat_k(const HeatArgs& a, const Geometry& g, cudaStream_t stream) {
   // at least half the shared memory of an SM, so that one CTA (with its 512
   // TMEM columns) is resident per SM whatever the register count
   const int smem = max(int(sizeof(HeatSmem<D>) + 1024), 116 * 1024);
-  cudaError_t e = cudaMemsetAsync(a.heat, 0, size_t(g.BH) * g.nb * g.nb * sizeof(float), stream);
+  cudaError_t e;
+  if (MAP) {
+    e = cudaMemsetAsync(a.heat, 0, size_t(g.BH) * g.nb * g.nb * sizeof(float), stream);
+    if (e != cudaSuccess) return e;
+  }
+  e = cudaFuncSetAttribute(heat_kernel<D, MAP, ENT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(heat_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  heat_kernel<D><<<unsigned(heat_ctas(g)), kHThreads, smem, stream>>>(a, g);
+  heat_kernel<D, MAP, ENT><<<unsigned(heat_ctas(g)), kHThreads, smem, stream>>>(a, g);
   return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_heat_d(const HeatArgs& a, const Geometry& g, cudaStream_t stream) {
+  if (a.heat != nullptr && a.entropy != nullptr) return launch_heat_k<D, true, true>(a, g, stream);
+  if (a.heat != nullptr) return launch_heat_k<D, true, false>(a, g, stream);
+  if (a.entropy != nullptr) return launch_heat_k<D, false, true>(a, g, stream);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_heat(const HeatArgs& a, const Geometry& g, cudaStream_t stream) {

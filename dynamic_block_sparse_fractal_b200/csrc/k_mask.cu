@@ -560,6 +560,10 @@ cudaError_t launch_mask(const MaskArgs& a, const Geometry& g, cudaStream_t strea
   else e = launch_select<96>(a, g, ld, stream);
   if (e != cudaSuccess) return e;
   if (marks != nullptr && (e = cudaEventRecord(marks[1], stream)) != cudaSuccess) return e;
+  return launch_union(a, g, stream);
+}
+
+cudaError_t launch_union(const MaskArgs& a, const Geometry& g, cudaStream_t stream) {
   const long items = long(g.BH) * g.ntile;
   const size_t warp_bytes = size_t(union_words_per_warp(g)) * sizeof(uint32_t);
   int wpc = int((48 * 1024) / warp_bytes);  // warps per CTA within 48 KB

@@ -43,6 +43,25 @@ struct MaskArgs {
 cudaError_t launch_mask(const MaskArgs& a, const Geometry& g, cudaStream_t stream,
                         cudaEvent_t* marks = nullptr);
 
+// Per-tile union lists from the rows' keep bitmaps (a.bits -> a.tcnt, a.tidx).
+cudaError_t launch_union(const MaskArgs& a, const Geometry& g, cudaStream_t stream);
+
+// Token Radius Attention block mask: per q-block row, the k-blocks that at
+// least vote_min of its query tokens reach (keep bitmap, count, ascending
+// list, as the select step writes them).
+struct RadiusArgs {
+  const float* entropy;  // [BH][S] natural order, nats
+  uint32_t* bits;        // [BH][nb][bitmap_words(g)]
+  int32_t* cnt;          // [BH][nb]
+  int32_t* idx;          // [BH][nb][nb]
+  float tau;             // keys per query = min(S, tau exp(H))
+  float gamma;           // radius decay exp(-gamma delta) per frame of distance
+  int vote_min;          // 1 .. N
+};
+cudaError_t launch_radius(const RadiusArgs& a, const Geometry& g, cudaStream_t stream);
+// The radius kernel's limits: T <= 4096 frames, Hh, Ww <= 1024, nb <= 6144 blocks.
+bool radius_supported(const Geometry& g);
+
 // Per head: tiles sorted by descending union length (ties by tile index).
 cudaError_t launch_tile_order(const int32_t* tcnt, int32_t* order, const Geometry& g,
                               cudaStream_t stream);
@@ -68,8 +87,10 @@ cudaError_t launch_attn(const AttnArgs& a, const Geometry& g, cudaStream_t strea
 // scratch).
 struct HeatArgs {
   CUtensorMap map_q, map_k;  // 5-D patch maps, one block per box
-  float* heat;               // [BH][nb][nb], fractal block order
-  float* scratch;            // [heat_ctas(g)][nb][256]
+  float* heat;               // [BH][nb][nb], fractal block order (null: no map)
+  float* scratch;            // [heat_ctas(g)][nb][256] (map only)
+  float* entropy;            // [BH][S] natural order: each query's attention entropy
+                             // in nats (null: none); heat or entropy must be given
   uint32_t* status;
   float scale_log2;  // log2(e) / sqrt(d)
   int debug_flags;   // SA_DEBUG_STALL_LOADER: the first K load is never issued (test hook)

@@ -360,6 +360,54 @@ sa_status sparse_attn_block_heatmap(const sa_desc* desc, const void* q, const vo
                                     void* workspace, size_t ws_bytes, float* heat,
                                     void* scratch, size_t scratch_bytes, void* stream);
 
+/* ---- Token Radius Attention mask (a second mask builder) -----------------
+ * "Token Radius Attention per la Generazione di Video Efficiente"
+ * (gist.science/it/paper/2608.02504), section 2, "La Pipeline TRA". Each query
+ * token gets a key budget from the entropy of its full attention row, the
+ * budget becomes a spatial radius that shrinks with the distance in frames,
+ * and token votes turn the per-token discs into a block mask in the same
+ * workspace format as sparse_attn_plan's, so that sparse_attn_fwd,
+ * sparse_attn_fwd_lse, sparse_attn_bwd and the graph calls run on it
+ * unchanged. */
+
+/* Step 1 ("Entropy-to-Budget", the dense warm-up): the entropy in nats of
+ * every query's full, unmasked attention row, H_i = -sum_j p_ij ln p_ij with
+ * p = softmax(q_i . k_j / sqrt(d)) over all keys, written to entropy: device
+ * fp32 [B*H][S] in natural token order, 4-byte aligned, owned by the caller.
+ * One dense pass (the cost of a dense Q K^T). q, k: as for sparse_attn_plan.
+ * workspace: as for sparse_attn_plan; only its status word is used (cleared
+ * on `stream` first, so sparse_attn_check reports this call). */
+sa_status sparse_attn_token_entropy(const sa_desc* desc, const void* q, const void* k,
+                                    void* workspace, size_t ws_bytes, float* entropy,
+                                    void* stream);
+
+typedef struct sa_radius {
+  float tau;     /* > 0: keys per query k_i = min(S, tau exp(H_i)) */
+  float gamma;   /* >= 0: the radius at a distance of delta frames is
+                    r_i exp(-gamma delta) */
+  int vote_min;  /* 1..N: query tokens of a q-block that must reach a k-block
+                    for the block pair to be kept */
+} sa_radius;
+
+/* Steps 2-3 ("Budget-to-Radius", "Kernel CUDA Fusi"): with
+ * Z(t) = sum over the frames t' of exp(-2 gamma |t' - t|) and r_i^2 =
+ * k_i / (pi Z(t_i)), key (t', h', w') is in query i's support iff
+ * (h' - h_i)^2 + (w' - w_i)^2 <= r_i^2 exp(-2 gamma |t' - t_i|) (token units);
+ * query i votes for a k-block iff its support holds one of the block's keys;
+ * q-block a keeps k-block b iff at least vote_min of its N queries vote for b.
+ * A query's own position is always in its support, so no row is empty.
+ * Writes the per-q-block lists, the per-tile union lists and the tile order
+ * into `workspace` exactly as sparse_attn_plan does (desc->thr and the STA
+ * window are not used; the pooled means are not written). entropy: device
+ * fp32 [B*H][S], natural order (e.g. from sparse_attn_token_entropy, possibly
+ * of an earlier step: the page reuses the warm-up entropies across steps).
+ * SA_ERR_INVALID_ARG for tau <= 0, gamma < 0, non-finite values or vote_min
+ * outside 1..N; SA_ERR_UNSUPPORTED beyond T = 4096 frames, Hh or Ww = 1024
+ * tokens, or 6144 blocks per head. */
+sa_status sparse_attn_plan_radius(const sa_desc* desc, const sa_radius* radius,
+                                  const float* entropy, void* workspace, size_t ws_bytes,
+                                  void* stream);
+
 #ifdef __cplusplus
 }
 #endif

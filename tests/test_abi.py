@@ -215,3 +215,22 @@ def test_plan_profile_names_and_rejection():
         api.SA_ERR_INVALID_ARG
     assert L.sparse_attn_plan_profile(ctypes.byref(d), FAKE, FAKE, FAKE, need, 0, us, 16,
                                       ctypes.byref(n), None) == api.SA_ERR_INVALID_ARG
+
+
+def test_radius_plan_rejects_bad_parameters_before_launch():
+    L = api.lib()
+    d = api.desc_for(W.TINY)
+    need = api.workspace_size(d)
+    for tau, gamma, vmin in ((0.0, 0.1, 1), (-1.0, 0.1, 1), (float("nan"), 0.1, 1),
+                             (1.0, -0.5, 1), (1.0, float("inf"), 1), (1.0, 0.1, 0),
+                             (1.0, 0.1, 65)):
+        r = api.SaRadius(tau, gamma, vmin)
+        assert L.sparse_attn_plan_radius(ctypes.byref(d), ctypes.byref(r), FAKE, FAKE, need,
+                                         None) == api.SA_ERR_INVALID_ARG, (tau, gamma, vmin)
+    r = api.SaRadius(1.0, 0.1, 1)
+    assert L.sparse_attn_plan_radius(ctypes.byref(d), ctypes.byref(r), None, FAKE, need,
+                                     None) == api.SA_ERR_INVALID_ARG
+    assert L.sparse_attn_plan_radius(ctypes.byref(d), ctypes.byref(r), FAKE, FAKE, need - 1,
+                                     None) == api.SA_ERR_WORKSPACE
+    assert L.sparse_attn_token_entropy(ctypes.byref(d), FAKE, FAKE, FAKE, need, None,
+                                       None) == api.SA_ERR_INVALID_ARG
