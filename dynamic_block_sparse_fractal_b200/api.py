@@ -56,7 +56,8 @@ class SaRadius(ctypes.Structure):
 class SaMaskViews(ctypes.Structure):
     _fields_ = [("qbar", ctypes.c_void_p), ("kbar", ctypes.c_void_p), ("cnt", ctypes.c_void_p),
                 ("idx", ctypes.c_void_p), ("tile_cnt", ctypes.c_void_p),
-                ("tile_idx", ctypes.c_void_p), ("nb", ctypes.c_int), ("ntile", ctypes.c_int)]
+                ("tile_idx", ctypes.c_void_p), ("nb", ctypes.c_int), ("ntile", ctypes.c_int),
+                ("logits", ctypes.c_void_p), ("logits_ld", ctypes.c_int)]
 
 
 class SparseAttnError(RuntimeError):
@@ -358,6 +359,8 @@ def get_mask(desc: SaDesc, workspace: torch.Tensor) -> dict:
         "idx": view(v.idx, BH * nb * nb, torch.int32, (BH, nb, nb)),
         "tile_cnt": view(v.tile_cnt, BH * nt, torch.int32, (BH, nt)),
         "tile_idx": view(v.tile_idx, BH * nt * nb, torch.int32, (BH, nt, nb)),
+        "logits": view(v.logits, BH * nb * v.logits_ld, torch.float32,
+                       (BH, nb, v.logits_ld))[:, :, :nb],
     }
 
 

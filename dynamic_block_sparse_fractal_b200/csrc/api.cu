@@ -14,10 +14,11 @@ using namespace sa;
 
 namespace {
 
-// Largest block count per head: the attention kernel stages a tile's union
-// list (<= nb entries) in shared memory sized for 2880 entries (the select
-// kernel's register-held rows would allow 3072).
-constexpr int kMaxBlocks = 2880;
+// Largest block count per head: the select kernel holds a row's masses in
+// shared memory up to 6144 (192 per lane), and the radius kernel's row
+// bitmap has 192 words. (The attention and gradient kernels stage the first
+// 2880 entries of a list in shared memory and read the rest from L2.)
+constexpr int kMaxBlocks = 6144;
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -414,6 +415,8 @@ sa_status sparse_attn_get_mask(const sa_desc* desc, const void* workspace, size_
   views->tile_idx = at<int32_t>(workspace, w.tidx);
   views->nb = g.nb;
   views->ntile = g.ntile;
+  views->logits = at<float>(workspace, w.logits);
+  views->logits_ld = logits_ld(g);
   return SA_OK;
 }
 

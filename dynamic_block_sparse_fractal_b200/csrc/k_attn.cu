@@ -59,7 +59,9 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // 7% slower and 2 of 8 17% slower (the softmax warps are limited by issue and
 // latency, not by the SFU's rate), so all go to the SFU.
 constexpr int kPolyPairsPer8 = 0;
-constexpr int kMaxList = 2880;             // largest union: nb <= 2880 blocks
+// Union entries staged in shared memory per tile; longer unions (heads of
+// more than 2880 blocks) read the rest from global memory (L2).
+constexpr int kMaxList = 2880;
 
 __host__ __device__ constexpr uint32_t col_s(int x) { return uint32_t(x) * 128u; }
 __host__ __device__ constexpr uint32_t col_o(int x) { return 256u + uint32_t(x) * 128u; }
@@ -83,8 +85,13 @@ struct Tile {
   int qa, qb;           // q-blocks (qb = -1: lone block)
   int n_u;              // union length
   int nsteps;           // ceil(n_u / 2)
-  const int32_t* list;  // union entries (shared-memory copy)
+  const int32_t* list;   // union entries (shared-memory copy of the first kMaxList)
+  const int32_t* glist;  // the same entries in global memory
 };
+
+__device__ __forceinline__ int list_at(const Tile& t, int i) {
+  return i < kMaxList ? t.list[i] : __ldg(t.glist + i);
+}
 
 // The MMA issue order shared by the loader and the MMA warp.
 struct OpIter {
@@ -164,14 +171,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     tile[x].qa = tile[x].qb = -1;
     tile[x].n_u = tile[x].nsteps = 0;
     tile[x].list = nullptr;
+    tile[x].glist = nullptr;
     if (pos < g.ntile) {
       const int t = a.order[size_t(bh) * g.ntile + pos];
       tile_blocks(g, t, tile[x].qa, tile[x].qb);
       tile[x].n_u = a.tcnt[size_t(bh) * g.ntile + t];
       tile[x].nsteps = (tile[x].n_u + 1) >> 1;
       const int32_t* src = a.tidx + (size_t(bh) * g.ntile + t) * g.nb;
+      tile[x].glist = src;
       // every warp reads the lists at each step: stage them in shared memory
-      for (int i = threadIdx.x; i < tile[x].n_u; i += kThreads) sm.list[x][i] = src[i];
+      const int staged = tile[x].n_u < kMaxList ? tile[x].n_u : kMaxList;
+      for (int i = threadIdx.x; i < staged; i += kThreads) sm.list[x][i] = src[i];
     }
     tile[x].list = sm.list[x];
   }
@@ -251,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Tile t = x ? tile[1] : tile[0];
         const int nblk = step_blocks(t, step);
         mbar_arrive_expect_tx(&sm.full[s], uint32_t(nblk) * 64u * D * 2u);
-        const int e0 = t.list[2 * step];
+        const int e0 = list_at(t, 2 * step);
         if (nblk == 2 && (e0 & kEntryTPair) && (e0 & kEntryBlockMask) + g.nh * g.nw < g.nb) {
           // the same patch in frames t, t+1: one two-frame box per channel half
           int tt, hp, wp;
@@ -262,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           const CUtensorMap* map = kind == 0 ? &a.map_k : &a.map_v;
           for (int e = 0; e < nblk; ++e) {
-            int kb = t.list[2 * step + e] & kEntryBlockMask;
+            int kb = list_at(t, 2 * step + e) & kEntryBlockMask;
             if (kb >= g.nb) {
               atomicOr(a.status, kDevErrBadIndex);
               kb = 0;
@@ -408,8 +418,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int j = 0; j < t.nsteps; ++j) {
       const int nblk = step_blocks(t, j);
-      const int e0 = t.list[2 * j];
-      const int e1 = nblk == 2 ? t.list[2 * j + 1] : 0;
+      const int e0 = list_at(t, 2 * j);
+      const int e1 = nblk == 2 ? list_at(t, 2 * j + 1) : 0;
       const bool keep0 = row_valid && (e0 & keep_bit);
       const bool keep1 = row_valid && nblk == 2 && (e1 & keep_bit);
       const int ks = s_op_index(x, j, tile[0].nsteps, tile[1].nsteps);

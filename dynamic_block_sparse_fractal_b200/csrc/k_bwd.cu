@@ -152,7 +152,9 @@ constexpr int kBChunk = 128 * 128;    // 128 rows x 128 B (64 bf16 channels)
 // (bf16 pairs) into the first 32 of them, so the two never write columns the
 // other still reads; the MMAs read P and dS as two K = 64 halves.
 constexpr uint32_t kColDV = 0, kColDK = 128, kColS = 256, kColDP = 384;
-constexpr int kBMaxEntries = 2880;  // the most blocks a head may have
+// List entries staged in shared memory per key tile; longer lists (heads of
+// more than 2880 blocks) read the rest from global memory (L2).
+constexpr int kBMaxEntries = 2880;
 
 template <int D>
 struct __align__(1024) BwdSmem {
@@ -227,7 +229,11 @@ __global__ void __launch_bounds__(kBThreads, 1)
   const int cnt = a.kcnt[unit];
   const int nsteps = (cnt + 1) / 2;
   // the key tile's list, read once (every role walks it step by step)
-  for (int i = threadIdx.x; i < cnt; i += kBThreads) sm.ent[i] = a.kidx[unit * g.nb + i];
+  const int32_t* gent = a.kidx + unit * g.nb;
+  for (int i = threadIdx.x; i < cnt && i < kBMaxEntries; i += kBThreads) sm.ent[i] = gent[i];
+  auto ent_at = [&](int i) -> int {
+    return i < kBMaxEntries ? sm.ent[i] : __ldg(gent + i);
+  };
   if (threadIdx.x == 0) {
     sm.abort = 0;
     mbar_init(&sm.kv_full, 1);
@@ -258,7 +264,6 @@ __global__ void __launch_bounds__(kBThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort = &sm.abort;
-  const int32_t* ent = sm.ent;
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA
@@ -285,8 +290,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
         const bool two = 2 * j + 1 < cnt;
         const int nq = two ? 2 : 1;
         int blk[2];
-        blk[0] = ent[2 * j] & kEntryBlockMask;
-        blk[1] = two ? (ent[2 * j + 1] & kEntryBlockMask) : blk[0];
+        blk[0] = ent_at(2 * j) & kEntryBlockMask;
+        blk[1] = two ? (ent_at(2 * j + 1) & kEntryBlockMask) : blk[0];
         // Q (two slots: loaded a step ahead)
         if (j >= 2 && !mbar_wait(&sm.q_empty[slot], ((j >> 1) - 1) & 1, abort)) {
           fail_b(a.status, &sm.abort, kDevErrTimeoutLoad);
@@ -431,7 +436,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
     for (int j = 0; j < nsteps; ++j) {
       const int slot = j & 1;
       const bool two = 2 * j + 1 < cnt;
-      const int f0 = ent[2 * j], f1 = two ? ent[2 * j + 1] : 0;
+      const int f0 = ent_at(2 * j), f1 = two ? ent_at(2 * j + 1) : 0;
       const bool mine = wg == 0 || two;                       // this half has a q-block
       const bool keep = mine && (((wg ? f1 : f0) & my_keep) != 0);  // uniform across the warp
       const float* lse2 = &sm.lse2[slot][64 * wg];

@@ -196,7 +196,26 @@ __global__ void __launch_bounds__(kLtThreads, 1)
 // ------------------------------------------------------------------ select
 constexpr int kSelWarps = 8;
 constexpr int kCandCap = 256;    // compacted search window per warp (8 per lane)
-constexpr int kMaxRowWords = 96;  // keep-bitmap words of a row (nb <= 3072)
+constexpr int kMaxRowWords = 192;  // keep-bitmap words of a row (nb <= 6144)
+constexpr int kRegVPL = 96;        // longest row held in registers (nb <= 3072)
+
+// A row's integer masses, VPL per lane (column j in lane j % 32, slot
+// j / 32): in registers, or, for rows too long for the register file, in the
+// warp's own shared-memory slice [VPL][32].
+template <int VPL, bool kSmem>
+struct RowStore;
+template <int VPL>
+struct RowStore<VPL, false> {
+  uint32_t v[VPL];
+  __device__ __forceinline__ uint32_t get(int i) const { return v[i]; }
+  __device__ __forceinline__ void set(int i, uint32_t x) { v[i] = x; }
+};
+template <int VPL>
+struct RowStore<VPL, true> {
+  uint32_t* p;  // this lane's column of the slice
+  __device__ __forceinline__ uint32_t get(int i) const { return p[i * 32]; }
+  __device__ __forceinline__ void set(int i, uint32_t x) { p[i * 32] = x; }
+};
 
 __device__ __forceinline__ uint32_t warp_sum_u32(uint32_t s) {
 #pragma unroll
@@ -206,14 +225,17 @@ __device__ __forceinline__ uint32_t warp_sum_u32(uint32_t s) {
 
 // Sum over the warp of the masses >= c; eight independent partial sums keep
 // the adds pipelined. (The sum of the masses > c is the one at c + 1.)
-template <int N>
-__device__ __forceinline__ uint32_t mass_at_least(const uint32_t (&m)[N], uint32_t c) {
+template <int N, class Store>
+__device__ __forceinline__ uint32_t mass_at_least(const Store& m, uint32_t c) {
   constexpr int kAcc = N < 8 ? N : 8;
   uint32_t acc[kAcc];
 #pragma unroll
   for (int i = 0; i < kAcc; ++i) acc[i] = 0u;
 #pragma unroll
-  for (int i = 0; i < N; ++i) acc[i % kAcc] += m[i] >= c ? m[i] : 0u;
+  for (int i = 0; i < N; ++i) {
+    const uint32_t x = m.get(i);
+    acc[i % kAcc] += x >= c ? x : 0u;
+  }
 #pragma unroll
   for (int w = 1; w < kAcc; w <<= 1)
 #pragma unroll
@@ -222,11 +244,13 @@ __device__ __forceinline__ uint32_t mass_at_least(const uint32_t (&m)[N], uint32
 }
 
 // VPL = values per lane: column j of the row sits in lane j % 32, slot j / 32.
-template <int VPL>
+// kSmem: the masses live in dynamic shared memory (VPL * 32 words per warp).
+template <int VPL, bool kSmem>
 __global__ void __launch_bounds__(kSelWarps * 32, VPL <= 32 ? 4 : (VPL <= 64 ? 2 : 1))
     select_kernel(const float* __restrict__ L, MaskArgs a, Geometry g, int ld) {
   __shared__ uint32_t cand_all[kSelWarps][kCandCap];
   __shared__ uint32_t rbits_all[kSelWarps][kMaxRowWords];
+  extern __shared__ uint32_t sel_slice[];  // kSmem only: [warp][VPL][32]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long row = long(blockIdx.x) * kSelWarps + warp;
   if (row >= long(g.BH) * g.nb) return;
@@ -236,15 +260,17 @@ __global__ void __launch_bounds__(kSelWarps * 32, VPL <= 32 ? 4 : (VPL <= 64 ? 2
   constexpr float kLog2e = 1.4426950408889634f;
 
   // ---- row softmax; each probability as an integer mass m = p * 2^30
-  uint32_t m[VPL];
+  // (the same operations, in the same order, whichever storage holds them)
+  RowStore<VPL, kSmem> m;
+  if constexpr (kSmem) m.p = sel_slice + size_t(warp) * VPL * 32 + lane;
   {
-    float v[VPL];
     float mx = -INFINITY;
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
       const int j = lane + 32 * i;
-      v[i] = j < nb ? __ldg(Lr + j) : -INFINITY;
-      mx = fmaxf(mx, v[i]);
+      const float v = j < nb ? __ldg(Lr + j) : -INFINITY;
+      m.set(i, __float_as_uint(v));
+      mx = fmaxf(mx, v);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
@@ -252,14 +278,16 @@ __global__ void __launch_bounds__(kSelWarps * 32, VPL <= 32 ? 4 : (VPL <= 64 ? 2
     float sum = 0.f;
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
-      v[i] = ex2_approx(fmaf(v[i], kLog2e, shift));  // exactly 0 in the padding slots
-      sum += v[i];
+      // exactly 0 in the padding slots
+      const float v = ex2_approx(fmaf(__uint_as_float(m.get(i)), kLog2e, shift));
+      m.set(i, __float_as_uint(v));
+      sum += v;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(kFull, sum, o);
     const float to_fx = 1073741824.0f / sum;  // 2^30 / sum
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) m[i] = __float2uint_rn(v[i] * to_fx);
+    for (int i = 0; i < VPL; ++i) m.set(i, __float2uint_rn(__uint_as_float(m.get(i)) * to_fx));
   }
 
   // ---- CDF threshold. In descending mass order (ties by index), block j is
@@ -289,7 +317,7 @@ __global__ void __launch_bounds__(kSelWarps * 32, VPL <= 32 ? 4 : (VPL <= 64 ? 2
         }
         uint32_t mmax = 0;
 #pragma unroll
-        for (int i = 0; i < VPL; ++i) mmax = max(mmax, m[i]);
+        for (int i = 0; i < VPL; ++i) mmax = max(mmax, m.get(i));
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mmax = max(mmax, __shfl_xor_sync(kFull, mmax, o));
         hi = 31 - __clz(mmax);  // G(2^lo) >= target holds for lo = 0
@@ -300,20 +328,20 @@ __global__ void __launch_bounds__(kSelWarps * 32, VPL <= 32 ? 4 : (VPL <= 64 ? 2
       } else if (stage == kAbove) {
         // the rest of the search over the compacted window only
         const uint32_t above = s;
-        uint32_t cw[kCandCap / 32];
+        RowStore<kCandCap / 32, false> cwr;
         const int wcnt = mid;
 #pragma unroll
         for (int k = 0; k < kCandCap / 32; ++k) {
           const int at = 32 * k + lane;
-          cw[k] = at < wcnt ? cand_all[warp][at] : 0u;  // 0 is below every candidate
+          cwr.set(k, at < wcnt ? cand_all[warp][at] : 0u);  // 0 is below every candidate
         }
 #pragma unroll 1
         for (; b >= 0; --b) {
           const uint32_t t = x | (1u << b);
-          if (above + mass_at_least<kCandCap / 32>(cw, t) >= tgt) x = t;
+          if (above + mass_at_least<kCandCap / 32>(cwr, t) >= tgt) x = t;
         }
         tau = x;
-        keep_ties = (tgt - above - mass_at_least<kCandCap / 32>(cw, tau + 1) + tau - 1) / tau;
+        keep_ties = (tgt - above - mass_at_least<kCandCap / 32>(cwr, tau + 1) + tau - 1) / tau;
         break;
       } else if (stage == kBits) {
         if (s >= tgt) x = c;
@@ -334,10 +362,11 @@ __global__ void __launch_bounds__(kSelWarps * 32, VPL <= 32 ? 4 : (VPL <= 64 ? 2
         int wcnt = 0;  // compact the window [x, 2x); order does not matter for sums
 #pragma unroll
         for (int i = 0; i < VPL; ++i) {
-          const bool in = (m[i] - x) < x;  // unsigned: x <= m < 2x
+          const uint32_t mi = m.get(i);
+          const bool in = (mi - x) < x;  // unsigned: x <= m < 2x
           const unsigned bal = __ballot_sync(kFull, in);
           const int at = wcnt + __popc(bal & lanemask_lt());
-          if (in && at < kCandCap) cand_all[warp][at] = m[i];
+          if (in && at < kCandCap) cand_all[warp][at] = mi;
           wcnt += __popc(bal);
         }
         __syncwarp();
@@ -369,8 +398,9 @@ __global__ void __launch_bounds__(kSelWarps * 32, VPL <= 32 ? 4 : (VPL <= 64 ? 2
   for (int i = 0; i < VPL; ++i) {
     if (32 * i < nb) {  // warp-uniform
       const bool valid = lane + 32 * i < nb;
-      bool nab = valid && (keep_all || m[i] > tau);
-      const bool tie = valid && !keep_all && m[i] == tau;
+      const uint32_t mi = m.get(i);
+      bool nab = valid && (keep_all || mi > tau);
+      const bool tie = valid && !keep_all && mi == tau;
       const unsigned tb = __ballot_sync(kFull, tie);
       if (tie) nab = (ties + __popc(tb & lanemask_lt())) < keep_ties;
       ties += __popc(tb);
@@ -526,8 +556,15 @@ __global__ void __launch_bounds__(kUnionMaxWarps * 32) union_kernel(MaskArgs a, 
 template <int VPL>
 cudaError_t launch_select(const MaskArgs& a, const Geometry& g, int ld, cudaStream_t stream) {
   const long rows = long(g.BH) * g.nb;
-  select_kernel<VPL><<<unsigned((rows + kSelWarps - 1) / kSelWarps), kSelWarps * 32, 0, stream>>>(
-      a.logits, a, g, ld);
+  constexpr bool kSmem = VPL > kRegVPL;
+  const size_t smem = kSmem ? size_t(kSelWarps) * VPL * 32 * sizeof(uint32_t) : 0;
+  if (kSmem) {
+    cudaError_t e = cudaFuncSetAttribute(select_kernel<VPL, kSmem>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+  }
+  select_kernel<VPL, kSmem><<<unsigned((rows + kSelWarps - 1) / kSelWarps), kSelWarps * 32, smem,
+                              stream>>>(a.logits, a, g, ld);
   return cudaGetLastError();
 }
 
@@ -551,13 +588,14 @@ cudaError_t launch_mask(const MaskArgs& a, const Geometry& g, cudaStream_t strea
                              : launch_logits<64>(a, g, ld, stream);
   if (e != cudaSuccess) return e;
   if (marks != nullptr && (e = cudaEventRecord(marks[0], stream)) != cudaSuccess) return e;
-  const int vpl = (g.nb + 31) / 32;  // nb <= 3072 (checked by the entry points)
+  const int vpl = (g.nb + 31) / 32;  // nb <= 6144 (checked by the entry points)
   if (vpl <= 4) e = launch_select<4>(a, g, ld, stream);
   else if (vpl <= 8) e = launch_select<8>(a, g, ld, stream);
   else if (vpl <= 16) e = launch_select<16>(a, g, ld, stream);
   else if (vpl <= 32) e = launch_select<32>(a, g, ld, stream);
   else if (vpl <= 64) e = launch_select<64>(a, g, ld, stream);
-  else e = launch_select<96>(a, g, ld, stream);
+  else if (vpl <= 96) e = launch_select<96>(a, g, ld, stream);
+  else e = launch_select<192>(a, g, ld, stream);
   if (e != cudaSuccess) return e;
   if (marks != nullptr && (e = cudaEventRecord(marks[1], stream)) != cudaSuccess) return e;
   return launch_union(a, g, stream);
@@ -579,7 +617,7 @@ cudaError_t launch_union(const MaskArgs& a, const Geometry& g, cudaStream_t stre
 // one head's K/V in L2.
 __global__ void __launch_bounds__(1024) tile_order_kernel(const int32_t* __restrict__ tcnt,
                                                           int32_t* __restrict__ order, Geometry g) {
-  __shared__ uint32_t key[2048];
+  __shared__ uint32_t key[4096];
   const int bh = blockIdx.x;
   int n = 1;
   while (n < g.ntile) n <<= 1;

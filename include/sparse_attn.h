@@ -80,7 +80,8 @@ typedef enum sa_status {
                                  range, even STA window, misaligned pointer */
   SA_ERR_UNSUPPORTED = 2,     /* valid but not implemented: d not in {64,128},
                                  N != 64, block shape not N tokens, grid not
-                                 divisible by the block shape */
+                                 divisible by the block shape, more than 6144
+                                 blocks per head, B*H above 65535 */
   SA_ERR_WORKSPACE = 3,       /* workspace smaller than
                                  sparse_attn_workspace_size() */
   SA_ERR_CUDA = 4,            /* a CUDA runtime call or launch failed */
@@ -161,6 +162,11 @@ typedef struct sa_mask_views {
                                ascending order) */
   int nb;                /* blocks per head */
   int ntile;             /* query tiles per head (pairs of q-blocks) */
+  const float* logits;   /* [B*H][nb][logits_ld] the reduced map's scaled
+                            logits Qbar Kbar^T / sqrt(d) as the plan computed
+                            them (fp32, before the row softmax); the first nb
+                            of each row are valid */
+  int logits_ld;         /* row pitch of logits, in floats */
 } sa_mask_views;
 
 sa_status sparse_attn_get_mask(const sa_desc* desc, const void* workspace,

@@ -6,9 +6,10 @@ ranked before it is < 1 - thr". That mass is uncertain in two ways:
 
   * the fp32 reduced map differs from the fp64 one by ~1e-6, so a block whose
     cumulative mass lies within MASK_BAND (1e-4) of 1 - thr may flip;
-  * blocks whose probabilities agree to within TIE_REL (relative) can be
-    ranked either way, so block j's cumulative mass is only known to lie in
-    [c_lo, c_hi], the mass of blocks surely above it vs. possibly above it.
+  * blocks whose probabilities agree to within the tie window (relative, per
+    row, from the measured logit error; see LOGIT_REL) can be ranked either
+    way, so block j's cumulative mass is only known to lie in [c_lo, c_hi],
+    the mass of blocks surely above it vs. possibly above it.
 
 A block is ambiguous when that interval, widened by MASK_BAND, straddles
 1 - thr. Blocks forced in by the STA window are never ambiguous. In addition,
@@ -27,7 +28,18 @@ import numpy as np
 import torch
 
 MASK_BAND = 1e-4
-TIE_REL = 1e-4
+# Ranking ties. The GPU's reduced-map logits carry an error of at most
+# 2.0e-6 of L1 = sum_c |qbar_c kbar_c| / sqrt(d) (measured on two heads each
+# of the HunyuanVideo-like, 8k and two scale-4 sweep workloads: three TF32
+# products of a hi/lo split, accumulated in fp32); LOGIT_REL doubles that. Two
+# probabilities of one row can then swap order only if their ratio is within
+# 2 * LOGIT_REL * (the row's largest L1) of 1, plus the fp32 exponential and
+# normalisation (EXP_REL), or if they differ by less than the 2^-30 mass
+# quantum the kernel ranks by (TIE_ABS).
+LOGIT_REL = 4e-6
+EXP_REL = 2.0 ** -21
+TIE_ABS = 2.0 ** -30
+TIE_REL = 1e-4  # the fallback when no pooled means are given
 OUT_MAX_ABS = 2e-2
 OUT_MEAN_ABS = 2e-3
 
@@ -42,19 +54,30 @@ def lists_to_mask(cnt: np.ndarray, idx: np.ndarray) -> np.ndarray:
     return m[..., :nb]
 
 
+def tie_rel_rows(qbar: np.ndarray, kbar: np.ndarray) -> np.ndarray:
+    """Per-row relative tie window from the pooled means of one or more
+    heads ([..., nb, d] each): 2 LOGIT_REL max_j L1[i, j] + EXP_REL."""
+    qa, ka = np.abs(qbar), np.abs(kbar)
+    L1 = np.matmul(qa, np.swapaxes(ka, -1, -2)) / np.sqrt(qbar.shape[-1])
+    return 2.0 * LOGIT_REL * L1.max(axis=-1) + EXP_REL
+
+
 def ambiguous(A: np.ndarray, thr: float, band: float = MASK_BAND,
-              rel: float = TIE_REL) -> np.ndarray:
-    """Bool mask of blocks whose keep decision the tolerances leave open."""
+              rel=TIE_REL) -> np.ndarray:
+    """Bool mask of blocks whose keep decision the tolerances leave open.
+    rel: a relative tie window, scalar or one per row (shape A.shape[:-1])."""
     if thr == 0.0:
         return np.zeros(A.shape, dtype=bool)
     shape = A.shape
     a = torch.from_numpy(np.ascontiguousarray(A.reshape(-1, shape[-1])))
+    r = torch.from_numpy(np.broadcast_to(np.asarray(rel, dtype=np.float64),
+                                         shape[:-1]).reshape(-1, 1).copy())
     asc, _ = torch.sort(a, dim=-1)
     n = a.shape[-1]
     top = torch.cumsum(torch.flip(asc, dims=[-1]), dim=-1)
     cs = torch.cat([torch.zeros(a.shape[0], 1, dtype=a.dtype), top], dim=-1)  # sum of k largest
-    n_gt = n - torch.searchsorted(asc, a * (1 + rel), right=True)
-    n_ge = n - torch.searchsorted(asc, a * (1 - rel), right=False)
+    n_gt = n - torch.searchsorted(asc, a * (1 + r) + TIE_ABS, right=True)
+    n_ge = n - torch.searchsorted(asc, a * (1 - r) - TIE_ABS, right=False)
     c_lo = torch.gather(cs, 1, n_gt)
     c_hi = torch.gather(cs, 1, n_ge) - a
     target = 1.0 - thr
@@ -64,10 +87,11 @@ def ambiguous(A: np.ndarray, thr: float, band: float = MASK_BAND,
 
 
 def compare_masks(gpu: np.ndarray, M: np.ndarray, M_nabla: np.ndarray, A: np.ndarray,
-                  thr: float) -> dict:
-    """Returns counts; 'bad' must be 0 and 'min_mass_margin' >= -MASK_BAND."""
+                  thr: float, rel=TIE_REL) -> dict:
+    """Returns counts; 'bad' must be 0 and 'min_mass_margin' >= -MASK_BAND.
+    rel: the tie window (tie_rel_rows of the heads' pooled means)."""
     sta_only = M & ~M_nabla
-    amb = ambiguous(A, thr) & ~sta_only
+    amb = ambiguous(A, thr, rel=rel) & ~sta_only
     mismatch = gpu != M
     bad = mismatch & ~amb
     kept_mass = (A * gpu).sum(-1)
