@@ -46,6 +46,19 @@
 
 namespace sa {
 
+// Timeline trace (a diagnostics build with -DSA_TRACE=1 only): clock64
+// stamps of one CTA's MMA issuer (per unit: wait start, operands ready,
+// issued) and of its eight softmax warps (per step: S seen, P arrived).
+#ifndef SA_TRACE
+#define SA_TRACE 0
+#endif
+#if SA_TRACE
+constexpr int kTraceUnits = 1300, kTraceSteps = 500;
+constexpr int kTraceSoftmax = 4096, kTraceWords = kTraceSoftmax + 8 * 2 * kTraceSteps;
+__device__ long long g_attn_trace[kTraceWords];
+__device__ int g_attn_trace_cta[2] = {100, 3};
+#endif
+
 namespace {
 
 constexpr int kThreads = 384;
@@ -163,6 +176,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y;
   const int pair = blockIdx.x;
+#if SA_TRACE
+  const bool tr = int(blockIdx.x) == g_attn_trace_cta[0] && int(blockIdx.y) == g_attn_trace_cta[1];
+  if (tr && threadIdx.x == 0) g_attn_trace[kTraceSoftmax - 1] = clock64();
+#endif
 
   Tile tile[2];
 #pragma unroll
@@ -319,6 +336,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = mbar_wait(&sm.q_full[0], 0, abort);
       if (ok && n1 > 0) ok = mbar_wait(&sm.q_full[1], 0, abort);
       int k = 0;  // op index (ring position)
+#if SA_TRACE
+      int tr_u = 0;
+#endif
       // S_X(step) = Q_X K^T into tile X's S columns, the K pair in slot s
       auto mma_s = [&](int x, int step, int s) {
         const uint64_t qd = x ? qdesc1 : qdesc0;
@@ -366,6 +386,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int nx = x ? n1 : n0;
           if (!ok || j >= nx) continue;
           const bool has_s = j + 1 < nx;
+#if SA_TRACE
+          const long long tr_t0 = clock64();
+#endif
           const int s_pv = k & (kSlots - 1), s_s = (k + 1) & (kSlots - 1);
           const uint32_t par_pv = (k / kSlots) & 1, par_s = ((k + 1) / kSlots) & 1;
           // one round trip for all three barriers; a bounded wait only for
@@ -379,6 +402,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                  ((ready & 4u) || !has_s || mbar_wait(&sm.full[s_s], par_s, abort));
             if (!ok) break;
           }
+#if SA_TRACE
+          const long long tr_t1 = clock64();
+#endif
           tc_fence_after_sync();  // P was written by the softmax threads
           mma_pv(x, j, s_pv);
           mma_commit(&sm.empty[s_pv]);
@@ -390,6 +416,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(&sm.o_final[x]);
             k += 1;
           }
+#if SA_TRACE
+          if (tr && tr_u < kTraceUnits) {
+            g_attn_trace[3 * tr_u] = tr_t0;
+            g_attn_trace[3 * tr_u + 1] = tr_t1;
+            g_attn_trace[3 * tr_u + 2] = clock64();
+          }
+          ++tr_u;
+#endif
         }
       }
       if (!ok) {
@@ -426,6 +460,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xFFFFFFFFu,
                       mbar_wait(&sm.empty[ks & (kSlots - 1)], (ks / kSlots) & 1, abort));
       if (!ok) break;
+#if SA_TRACE
+      if (tr && lane == 0 && j < kTraceSteps)
+        g_attn_trace[kTraceSoftmax + (warp - 4) * 2 * kTraceSteps + 2 * j] = clock64();
+#endif
       tc_fence_after_sync();
       // keep0 / keep1 are uniform across a warp (a warp's rows lie in one
       // q-block), so the warp-collective loads may be skipped per block
@@ -508,6 +546,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_st();
       tc_fence_before_sync();
       mbar_arrive(&sm.p_full[x]);
+#if SA_TRACE
+      if (tr && lane == 0 && j < kTraceSteps)
+        g_attn_trace[kTraceSoftmax + (warp - 4) * 2 * kTraceSteps + 2 * j + 1] = clock64();
+#endif
     }
     if (t.nsteps > 0) {
       if (!ok) {
@@ -593,3 +635,17 @@ cudaError_t launch_attn(const AttnArgs& a, const Geometry& g, cudaStream_t strea
 }
 
 }  // namespace sa
+
+#if SA_TRACE
+// Diagnostics build only: choose the traced CTA, read the stamps back.
+extern "C" int sparse_attn_trace_select(int bx, int by) {
+  const int v[2] = {bx, by};
+  long long zero[sa::kTraceWords] = {};
+  if (cudaMemcpyToSymbol(sa::g_attn_trace, zero, sizeof(zero)) != cudaSuccess) return 1;
+  return cudaMemcpyToSymbol(sa::g_attn_trace_cta, v, sizeof(v)) != cudaSuccess;
+}
+extern "C" int sparse_attn_trace_read(long long* dst, int n) {
+  if (n > sa::kTraceWords) n = sa::kTraceWords;
+  return cudaMemcpyFromSymbol(dst, sa::g_attn_trace, sizeof(long long) * n) != cudaSuccess;
+}
+#endif

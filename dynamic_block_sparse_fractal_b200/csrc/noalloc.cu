@@ -16,20 +16,28 @@ constexpr int kMaxDevices = 64;
 // One copy per GPU that loads this library, held until the process exits.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
-// Device addresses of g_noalloc_scratch, looked up once per device. In host
-// code the symbol itself is only a host-side handle, never a device address.
+// Device addresses of g_noalloc_scratch per device. In host code the symbol
+// itself is only a host-side handle, never a device address. The address is
+// looked up again on every call made outside stream capture (a device reset
+// reloads the module, and the array may then sit elsewhere); a call made
+// while its stream is being captured cannot look it up and uses the address
+// the last uncaptured call on that device found.
 void* g_scratch_ptr[kMaxDevices] = {};
 std::mutex g_scratch_mu;
 
-sa_status scratch_for_current_device(void** out) {
+sa_status scratch_for_current_device(cudaStream_t stream, void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SA_ERR_CUDA;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return SA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
+  if (cap == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
       return SA_ERR_CUDA;
     g_scratch_ptr[dev] = p;
+  } else if (g_scratch_ptr[dev] == nullptr) {
+    return SA_ERR_CUDA;  // first call on this device inside a capture
   }
   *out = g_scratch_ptr[dev];
   return SA_OK;
@@ -45,7 +53,7 @@ extern "C" sa_status sparse_attn_forward_noalloc(const sa_desc* desc, const void
   if (st != SA_OK) return st;
   if (need > kScratchBytes) return SA_ERR_WORKSPACE;
   void* ws = nullptr;
-  st = scratch_for_current_device(&ws);
+  st = scratch_for_current_device(static_cast<cudaStream_t>(stream), &ws);
   if (st != SA_OK) return st;
   st = sparse_attn_plan(desc, q, k, ws, kScratchBytes, stream);
   if (st != SA_OK) return st;

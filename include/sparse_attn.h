@@ -206,8 +206,13 @@ const char* sparse_attn_status_string(sa_status status);
  * Returns SA_ERR_WORKSPACE, before launching anything, when the problem's
  * workspace (sparse_attn_workspace_size) is larger than the built-in array.
  *
- * - The first call on a device (with that device current) looks the array's
- *   device address up once; make that first call before any stream capture.
+ * - Every call made outside stream capture looks the array's device address
+ *   up (with the call's device current), so a device reset, which reloads
+ *   the library's device image, is followed safely. A call made while its
+ *   stream is being captured cannot look it up: it uses the address the last
+ *   uncaptured call on that device found, so make one uncaptured call on the
+ *   device first (and again after any device reset); otherwise it returns
+ *   SA_ERR_CUDA.
  * - All calls on a device share the one array, which keeps the previous
  *   call's contents (the plan rewrites everything it later reads). Calls whose
  *   work may overlap on the GPU (different streams, or several threads)
