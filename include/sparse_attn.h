@@ -100,7 +100,9 @@ sa_status sparse_attn_workspace_size(const sa_desc* desc, size_t* bytes);
  *   2. Qbar, Kbar = mean of the N tokens of each block, fp32 (Metodologia 2,
  *      "Sottocampionamento");
  *   3. A = row softmax(Qbar Kbar^T / sqrt(d)) (Metodologia 2, "Attenzione
- *      Ridotta"), never materialised;
+ *      Ridotta"); the scaled logits are written to the workspace (fp32,
+ *      nb x nb per head) and read back once by the threshold step, which
+ *      needs a whole row at a time;
  *   4. per row, k-block j is kept iff the mass of the blocks ranked before it
  *      (descending probability, ties by ascending index) is below 1 - thr
  *      (Metodologia 2, "CDF Thresholding"); thr == 0 keeps every block;
