@@ -69,12 +69,15 @@ def kept_flops_per_pair(w):
 
 
 # DRAM bytes (read + write) of one attention launch on the HunyuanVideo-like
-# workload, from the one-pass ncu capture of this kernel. Reported only while
-# the attention kernel's sources are the ones that capture measured.
+# workload: the ncu capture of this kernel on the same grid with 2 of the 24
+# heads (384.5 MB read + 56.1 MB written per launch), scaled by the 12 times
+# more heads (every head's tiles run in the same order, so per-head traffic is
+# the same). Reported only while the attention kernel's sources are the ones
+# that capture measured.
 ATTN_TRAFFIC = {
     "workload": "hunyuan_1x24x126720x128",
-    "bytes": 5.283e9 + 0.864e9,
-    "sources_sha1": "868fb496c3fe03a82886b2c5c9dfd3873585629e",
+    "bytes": 12 * (384.546560e6 + 56.089088e6),
+    "sources_sha1": "7baed63701d00a72c1b8b1da8c994391f79cc9cc",
 }
 ATTN_SOURCES = ("k_attn.cu", "sm100.cuh", "exp2_poly.cuh", "layout.cuh")
 
