@@ -195,9 +195,15 @@ __global__ void __launch_bounds__(kLtThreads, 1)
 
 // ------------------------------------------------------------------ select
 constexpr int kSelWarps = 8;
-constexpr int kCandCap = 256;    // compacted search window per warp (8 per lane)
+constexpr int kCandCap = 256;      // compacted search window per warp (8 per lane)
 constexpr int kMaxRowWords = 192;  // keep-bitmap words of a row (nb <= 6144)
 constexpr int kRegVPL = 96;        // longest row held in registers (nb <= 3072)
+// Per-warp shared work area, used in turn by the leading-bit histogram
+// (32 buckets x 32 lanes), the compacted window (words 0..255) and the keep
+// bitmap (words 256..447).
+constexpr int kSelWork = 32 * 32;
+constexpr int kRbitsAt = kCandCap;
+static_assert(kRbitsAt + kMaxRowWords <= kSelWork, "select work area");
 
 // A row's integer masses, VPL per lane (column j in lane j % 32, slot
 // j / 32): in registers, or, for rows too long for the register file, in the
@@ -217,12 +223,6 @@ struct RowStore<VPL, true> {
   __device__ __forceinline__ void set(int i, uint32_t x) { p[i * 32] = x; }
 };
 
-__device__ __forceinline__ uint32_t warp_sum_u32(uint32_t s) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(kFull, s, o);
-  return s;
-}
-
 // Sum over the warp of the masses >= c; eight independent partial sums keep
 // the adds pipelined. (The sum of the masses > c is the one at c + 1.)
 template <int N, class Store>
@@ -240,7 +240,7 @@ __device__ __forceinline__ uint32_t mass_at_least(const Store& m, uint32_t c) {
   for (int w = 1; w < kAcc; w <<= 1)
 #pragma unroll
     for (int i = 0; i + w < kAcc; i += 2 * w) acc[i] += acc[i + w];
-  return warp_sum_u32(acc[0]);
+  return __reduce_add_sync(kFull, acc[0]);
 }
 
 // VPL = values per lane: column j of the row sits in lane j % 32, slot j / 32.
@@ -248,8 +248,7 @@ __device__ __forceinline__ uint32_t mass_at_least(const Store& m, uint32_t c) {
 template <int VPL, bool kSmem>
 __global__ void __launch_bounds__(kSelWarps * 32, VPL <= 32 ? 4 : (VPL <= 64 ? 2 : 1))
     select_kernel(const float* __restrict__ L, MaskArgs a, Geometry g, int ld) {
-  __shared__ uint32_t cand_all[kSelWarps][kCandCap];
-  __shared__ uint32_t rbits_all[kSelWarps][kMaxRowWords];
+  __shared__ __align__(16) uint32_t work_all[kSelWarps][kSelWork];
   extern __shared__ uint32_t sel_slice[];  // kSmem only: [warp][VPL][32]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long row = long(blockIdx.x) * kSelWarps + warp;
@@ -257,6 +256,7 @@ __global__ void __launch_bounds__(kSelWarps * 32, VPL <= 32 ? 4 : (VPL <= 64 ? 2
   const int nb = g.nb;
   const int qb = int(row % nb);
   const float* Lr = L + size_t(row) * ld;
+  uint32_t* work = work_all[warp];
   constexpr float kLog2e = 1.4426950408889634f;
 
   // ---- row softmax; each probability as an integer mass m = p * 2^30
@@ -293,119 +293,121 @@ __global__ void __launch_bounds__(kSelWarps * 32, VPL <= 32 ? 4 : (VPL <= 64 ? 2
   // ---- CDF threshold. In descending mass order (ties by index), block j is
   // kept iff the mass ranked before it is < target. tau, the mass of the last
   // kept block, is the largest x with G(x) = (sum of the masses >= x) >=
-  // target; G does not increase with x. Found as: the leading bit e of tau
-  // by a binary search over bit positions, then the lower bits one by one.
-  // Once e is known only the masses in [2^e, 2^(e+1)) can still move G, so
-  // those (if few) are compacted to shared memory and searched alone, the
-  // masses >= 2^(e+1) entering as a constant. Blocks with mass > tau are
-  // kept, and of those with mass == tau the first
-  // ceil((target - G(tau + 1)) / tau) in index order. Every pass over the
-  // whole row goes through the one loop below (the code stays small).
+  // target; G does not increase with x, so tau is one of the masses.
+  //  1. The leading bit e of tau from one histogram of the masses by leading
+  //     bit (each lane adds into its own column of a 32 x 32 table; lane b
+  //     then sums row b, and a suffix scan over the lanes gives G(2^b) in
+  //     lane b): e is the highest b with G(2^b) >= target, and G(2^(e+1)),
+  //     the mass above the window [2^e, 2^(e+1)), comes with it.
+  //  2. The window's masses are compacted to shared memory (if at most 256)
+  //     and the lower bits of tau found one by one over them alone, the mass
+  //     above the window entering as a constant; a longer window is searched
+  //     bit by bit over the whole row.
+  // Blocks with mass > tau are kept, and of those with mass == tau the first
+  // ceil((target - G(tau + 1)) / tau) in index order.
   bool keep_all = a.dense != 0;
-  uint32_t tau = 0, keep_ties = 0;
+  uint32_t tau = 0, keep_ties = 0, n_tau = 0;  // n_tau: masses equal to tau (0: not counted)
   if (!keep_all) {
     const uint32_t tgt = a.target_fx;
-    enum { kTotal, kLead, kAbove, kBits, kTies };
-    int stage = kTotal, lo = 0, hi = 0, mid = 0, b = 0;
-    uint32_t c = 1u, x = 0u;
-    for (;;) {
-      const uint32_t s = mass_at_least<VPL>(m, c);
-      if (stage == kTotal) {
-        if (s < tgt) {  // total mass below the target (rounding): keep all
-          keep_all = true;
-          break;
-        }
-        uint32_t mmax = 0;
+    uint4* work4 = reinterpret_cast<uint4*>(work);
 #pragma unroll
-        for (int i = 0; i < VPL; ++i) mmax = max(mmax, m.get(i));
+    for (int k = lane; k < kSelWork / 4; k += 32) work4[k] = make_uint4(0u, 0u, 0u, 0u);
+    __syncwarp();
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mmax = max(mmax, __shfl_xor_sync(kFull, mmax, o));
-        hi = 31 - __clz(mmax);  // G(2^lo) >= target holds for lo = 0
-        stage = kLead;
-      } else if (stage == kLead) {
-        if (s >= tgt) lo = mid;
-        else hi = mid - 1;
-      } else if (stage == kAbove) {
-        // the rest of the search over the compacted window only
-        const uint32_t above = s;
+    for (int i = 0; i < VPL; ++i) {
+      const uint32_t mi = m.get(i);
+      if (mi != 0u) atomicAdd(work + (31 - __clz(mi)) * 32 + lane, mi);
+    }
+    __syncwarp();
+    uint32_t gs = 0;  // this lane's row; four words per load, the loads of a
+                      // quarter-warp on distinct banks
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      const uint4 q = work4[lane * 8 + ((lane + s) & 7)];
+      gs += (q.x + q.y) + (q.z + q.w);
+    }
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_down_sync(kFull, gs, o);
+      if (lane + o < 32) gs += t;
+    }
+    // lane b: G(2^b); lane 0: the total (masses are < 2^31, so lane 31: 0)
+    const uint32_t total = __shfl_sync(kFull, gs, 0);
+    __syncwarp();  // the table is read before the window overwrites it
+    if (total < tgt) {  // total mass below the target (rounding): keep all
+      keep_all = true;
+    } else {
+      const int e = 31 - __clz(__ballot_sync(kFull, gs >= tgt));
+      const uint32_t above = __shfl_sync(kFull, gs, e + 1);
+      uint32_t x = 1u << e;
+      int wcnt = 0;  // compact the window [x, 2x); order does not matter for sums
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const uint32_t mi = m.get(i);
+        const bool in = (mi - x) < x;  // unsigned: x <= m < 2x
+        const unsigned bal = __ballot_sync(kFull, in);
+        const int at = wcnt + __popc(bal & lanemask_lt());
+        if (in && at < kCandCap) work[at] = mi;
+        wcnt += __popc(bal);
+      }
+      __syncwarp();
+      if (wcnt <= kCandCap) {
         RowStore<kCandCap / 32, false> cwr;
-        const int wcnt = mid;
 #pragma unroll
         for (int k = 0; k < kCandCap / 32; ++k) {
           const int at = 32 * k + lane;
-          cwr.set(k, at < wcnt ? cand_all[warp][at] : 0u);  // 0 is below every candidate
+          cwr.set(k, at < wcnt ? work[at] : 0u);  // 0 is below every candidate
         }
 #pragma unroll 1
-        for (; b >= 0; --b) {
+        for (int b = e - 1; b >= 0; --b) {
           const uint32_t t = x | (1u << b);
           if (above + mass_at_least<kCandCap / 32>(cwr, t) >= tgt) x = t;
         }
         tau = x;
-        keep_ties = (tgt - above - mass_at_least<kCandCap / 32>(cwr, tau + 1) + tau - 1) / tau;
-        break;
-      } else if (stage == kBits) {
-        if (s >= tgt) x = c;
-        --b;
-      } else {  // kTies: s = G(tau + 1)
-        keep_ties = (tgt - s + tau - 1) / tau;
-        break;
-      }
-      // the next threshold
-      if (stage == kLead) {
-        if (lo < hi) {
-          mid = (lo + hi + 1) >> 1;
-          c = 1u << mid;
-          continue;
-        }
-        x = 1u << lo;
-        b = lo - 1;
-        int wcnt = 0;  // compact the window [x, 2x); order does not matter for sums
+        uint32_t eq = 0;
 #pragma unroll
-        for (int i = 0; i < VPL; ++i) {
-          const uint32_t mi = m.get(i);
-          const bool in = (mi - x) < x;  // unsigned: x <= m < 2x
-          const unsigned bal = __ballot_sync(kFull, in);
-          const int at = wcnt + __popc(bal & lanemask_lt());
-          if (in && at < kCandCap) cand_all[warp][at] = mi;
-          wcnt += __popc(bal);
-        }
-        __syncwarp();
-        if (wcnt <= kCandCap) {
-          mid = wcnt;
-          c = x << 1;
-          stage = kAbove;
-          continue;
-        }
-        stage = kBits;
-      }
-      if (stage == kBits) {
-        if (b >= 0) {
-          c = x | (1u << b);
-          continue;
+        for (int k = 0; k < kCandCap / 32; ++k) eq += cwr.get(k) == tau ? 1u : 0u;
+        n_tau = __reduce_add_sync(kFull, eq);
+        keep_ties = (tgt - above - mass_at_least<kCandCap / 32>(cwr, tau + 1) + tau - 1) / tau;
+      } else {
+#pragma unroll 1
+        for (int b = e - 1; b >= 0; --b) {
+          const uint32_t t = x | (1u << b);
+          if (mass_at_least<VPL>(m, t) >= tgt) x = t;
         }
         tau = x;
-        c = tau + 1u;
-        stage = kTies;
+        keep_ties = (tgt - mass_at_least<VPL>(m, tau + 1) + tau - 1) / tau;
       }
     }
   }
 
   // ---- keep bitmap in shared memory: the NABLA bits by ballot (ties in
-  // index order), then OR the STA box, clipped to the grid
-  uint32_t* rbits = rbits_all[warp];
-  uint32_t ties = 0;
+  // index order, unless every mass equal to tau is kept), then OR the STA
+  // box, clipped to the grid. Padding slots hold mass 0 < tau.
+  uint32_t* rbits = work + kRbitsAt;
+  if (keep_all || n_tau == keep_ties) {
 #pragma unroll
-  for (int i = 0; i < VPL; ++i) {
-    if (32 * i < nb) {  // warp-uniform
-      const bool valid = lane + 32 * i < nb;
-      const uint32_t mi = m.get(i);
-      bool nab = valid && (keep_all || mi > tau);
-      const bool tie = valid && !keep_all && mi == tau;
-      const unsigned tb = __ballot_sync(kFull, tie);
-      if (tie) nab = (ties + __popc(tb & lanemask_lt())) < keep_ties;
-      ties += __popc(tb);
-      const unsigned kb = __ballot_sync(kFull, nab);
-      if (lane == 0) rbits[i] = kb;
+    for (int i = 0; i < VPL; ++i) {
+      if (32 * i < nb) {  // warp-uniform
+        const bool nab = keep_all ? lane + 32 * i < nb : m.get(i) >= tau;
+        const unsigned kb = __ballot_sync(kFull, nab);
+        if (lane == 0) rbits[i] = kb;
+      }
+    }
+  } else {
+    uint32_t ties = 0;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      if (32 * i < nb) {  // warp-uniform
+        const uint32_t mi = m.get(i);
+        bool nab = mi > tau;
+        const bool tie = mi == tau;
+        const unsigned tb = __ballot_sync(kFull, tie);
+        if (tie) nab = (ties + __popc(tb & lanemask_lt())) < keep_ties;
+        ties += __popc(tb);
+        const unsigned kb = __ballot_sync(kFull, nab);
+        if (lane == 0) rbits[i] = kb;
+      }
     }
   }
   __syncwarp();
