@@ -46,25 +46,35 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 // ------------------------------------------------------------------ logits
 // L = Qbar Kbar^T / sqrt(d) per head on the TF32 tensor cores, in three
 // products of the pooled means' hi / lo split (hi*hi + hi*lo + lo*hi), fp32
-// accumulation in TMEM. One CTA per 128 x 256 output tile: warp 0 loads
-// 32-channel K-chunks of the four operands by TMA into a 2-stage ring, warp
-// 1 issues the MMAs (M=128, N=256, K=8), warps 2-5 read the accumulator,
-// scale it and store whole rows (staged through shared memory so the global
-// stores are coalesced).
+// accumulation in TMEM. A persistent kernel, one CTA per SM, walks the
+// 128 x 256 output tiles (column tiles fastest, so neighbouring CTAs share
+// the query rows in L2): warp 0 loads 32-channel K-chunks of the four
+// operands by TMA into a 2-stage ring, warp 1 issues the MMAs (M=128, N=256,
+// K=8) into one of two TMEM accumulators, and warps 2-5 read the other one,
+// scale it and store it (staged through shared memory, 32 x 32 per warp, so
+// that the global stores are whole 128-byte rows) while the next tile's
+// products run.
 constexpr int kLtM = 128, kLtN = 256, kLtK = 32;  // tile rows, columns, K-chunk (128 B of fp32)
 constexpr int kLtThreads = 192;
-constexpr int kLtStagePitch = kLtN + 4;  // floats per staged output row (conflict-free)
+constexpr int kLtStagePitch = 36;  // floats per staged 32-column row (float4 stores conflict-free)
 constexpr uint32_t kLtStageBytes = 2u * kLtM * kLtK * 4u + 2u * kLtN * kLtK * 4u;  // 96 KB
 
 struct __align__(1024) LogitsSmem {
   float a[2][2][kLtM * kLtK];  // [stage][hi, lo]: 128 rows x 128 B, 128-byte swizzle
   float b[2][2][kLtN * kLtK];  // [stage][hi, lo]: 256 rows x 128 B
-  uint64_t full[2], empty[2], acc_full;
+  float out[4][32 * kLtStagePitch];  // per epilogue warp: 32 rows x 32 columns
+  uint64_t full[2], empty[2], acc_full[2], acc_empty[2], drain;
   uint32_t tmem_base;
   int abort;
 };
-static_assert(4 * 32 * kLtStagePitch * 4 <= sizeof(float) * 2 * 2 * (kLtM + kLtN) * kLtK,
-              "the output staging reuses the operand stages");
+
+struct LtTile {
+  int bh, r0, c0;
+};
+__device__ __forceinline__ LtTile lt_tile(int t, int nrt, int nct) {
+  const int ct = t % nct, rest = t / nct;
+  return {rest / nrt, (rest % nrt) * kLtM, ct * kLtN};
+}
 
 template <int D>
 __global__ void __launch_bounds__(kLtThreads, 1)
@@ -74,20 +84,21 @@ __global__ void __launch_bounds__(kLtThreads, 1)
       (reinterpret_cast<uintptr_t>(lt_raw) + 1023) & ~uintptr_t(1023));
   constexpr int kChunks = D / kLtK;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.z;
-  const int r0 = blockIdx.y * kLtM, c0 = blockIdx.x * kLtN;
-  const int row_base = bh * g.nb;  // first row of this head in the [BH*nb][d] operands
+  const int nrt = (g.nb + kLtM - 1) / kLtM, nct = ld / kLtN;
+  const int ntiles = g.BH * nrt * nct;
   if (threadIdx.x == 0) {
     sm.abort = 0;
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], 1);
+      mbar_init(&sm.acc_full[s], 1);
+      mbar_init(&sm.acc_empty[s], 4);  // one arrival per epilogue warp
     }
-    mbar_init(&sm.acc_full, 1);
+    mbar_init(&sm.drain, 1);
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(&sm.tmem_base, 256);
+    tmem_alloc(&sm.tmem_base, 512);
     tmem_relinquish();
   }
   tc_fence_before_sync();
@@ -102,20 +113,24 @@ __global__ void __launch_bounds__(kLtThreads, 1)
       prefetch_tensormap(&a.map_qlo);
       prefetch_tensormap(&a.map_khi);
       prefetch_tensormap(&a.map_klo);
-      int issued = -1;
-      for (int c = 0; c < kChunks; ++c) {
-        const int s = c & 1;
-        if (c >= 2 && !mbar_wait(&sm.empty[s], ((c >> 1) - 1) & 1, abort)) {
-          fail_status(a.status, &sm.abort, kDevErrTimeoutLoad);
-          break;
+      int q = 0, issued = -1;  // chunks over this CTA's tiles
+      for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x) {
+        const LtTile tl = lt_tile(t, nrt, nct);
+        const int row_base = tl.bh * g.nb;  // first row of this head in the [BH*nb][d] operands
+        for (int c = 0; c < kChunks; ++c, ++q) {
+          const int s = q & 1;
+          if (q >= 2 && !mbar_wait(&sm.empty[s], ((q >> 1) - 1) & 1, abort)) {
+            if (!*abort) fail_status(a.status, &sm.abort, kDevErrTimeoutLoad);
+            break;
+          }
+          if (*abort) break;
+          mbar_arrive_expect_tx(&sm.full[s], kLtStageBytes);
+          tma_load_2d(sm.a[s][0], &a.map_qhi, &sm.full[s], c * kLtK, row_base + tl.r0);
+          tma_load_2d(sm.a[s][1], &a.map_qlo, &sm.full[s], c * kLtK, row_base + tl.r0);
+          tma_load_2d(sm.b[s][0], &a.map_khi, &sm.full[s], c * kLtK, row_base + tl.c0);
+          tma_load_2d(sm.b[s][1], &a.map_klo, &sm.full[s], c * kLtK, row_base + tl.c0);
+          issued = q;
         }
-        if (*abort) break;
-        mbar_arrive_expect_tx(&sm.full[s], kLtStageBytes);
-        tma_load_2d(sm.a[s][0], &a.map_qhi, &sm.full[s], c * kLtK, row_base + r0);
-        tma_load_2d(sm.a[s][1], &a.map_qlo, &sm.full[s], c * kLtK, row_base + r0);
-        tma_load_2d(sm.b[s][0], &a.map_khi, &sm.full[s], c * kLtK, row_base + c0);
-        tma_load_2d(sm.b[s][1], &a.map_klo, &sm.full[s], c * kLtK, row_base + c0);
-        issued = c;
       }
       if (*abort) {  // let this thread's copies land before the CTA can exit
         int never = 0;
@@ -127,70 +142,88 @@ __global__ void __launch_bounds__(kLtThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_tf32_f32(kLtM, kLtN);
       bool ok = true;
-      for (int c = 0; c < kChunks && ok; ++c) {
-        const int s = c & 1;
-        ok = mbar_wait(&sm.full[s], (c >> 1) & 1, abort);
+      int q = 0, i = 0;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++i) {
+        const int buf = i & 1;
+        if (i >= 2) ok = mbar_wait(&sm.acc_empty[buf], ((i >> 1) - 1) & 1, abort);
         if (!ok) break;
         tc_fence_after_sync();
-        const uint64_t ahi = sw128_desc(smem_u32(sm.a[s][0]), 16, 1024);
-        const uint64_t alo = sw128_desc(smem_u32(sm.a[s][1]), 16, 1024);
-        const uint64_t bhi = sw128_desc(smem_u32(sm.b[s][0]), 16, 1024);
-        const uint64_t blo = sw128_desc(smem_u32(sm.b[s][1]), 16, 1024);
+        const uint32_t acc = tmem + uint32_t(buf * kLtN);
+        for (int c = 0; c < kChunks; ++c, ++q) {
+          const int s = q & 1;
+          ok = mbar_wait(&sm.full[s], (q >> 1) & 1, abort);
+          if (!ok) break;
+          tc_fence_after_sync();
+          const uint64_t ahi = sw128_desc(smem_u32(sm.a[s][0]), 16, 1024);
+          const uint64_t alo = sw128_desc(smem_u32(sm.a[s][1]), 16, 1024);
+          const uint64_t bhi = sw128_desc(smem_u32(sm.b[s][0]), 16, 1024);
+          const uint64_t blo = sw128_desc(smem_u32(sm.b[s][1]), 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < kLtK / 8; ++kk) {  // K = 8 tf32 = 32 B per MMA
-          const uint32_t off = uint32_t(kk) * 2u;  // 32 B in 16-byte units
-          mma_tf32_ss(tmem, ahi + off, bhi + off, idesc, (c | kk) != 0 ? 1u : 0u);
-          mma_tf32_ss(tmem, ahi + off, blo + off, idesc, 1u);
-          mma_tf32_ss(tmem, alo + off, bhi + off, idesc, 1u);
+          for (int kk = 0; kk < kLtK / 8; ++kk) {  // K = 8 tf32 = 32 B per MMA
+            const uint32_t off = uint32_t(kk) * 2u;  // 32 B in 16-byte units
+            mma_tf32_ss(acc, ahi + off, bhi + off, idesc, (c | kk) != 0 ? 1u : 0u);
+            mma_tf32_ss(acc, ahi + off, blo + off, idesc, 1u);
+            mma_tf32_ss(acc, alo + off, bhi + off, idesc, 1u);
+          }
+          mma_commit(&sm.empty[s]);
         }
-        mma_commit(&sm.empty[s]);
+        if (ok) mma_commit(&sm.acc_full[buf]);
       }
-      if (ok) {
-        mma_commit(&sm.acc_full);
-      } else {
-        fail_status(a.status, &sm.abort, kDevErrTimeoutMma);
-        mma_commit(&sm.acc_full);  // lets the epilogue and the CTA end (bounded)
-        int never = 0;
-        mbar_wait(&sm.acc_full, 0, &never);
-      }
+      if (!ok && !*abort) fail_status(a.status, &sm.abort, kDevErrTimeoutMma);
+      // no MMA of this thread may be in flight when the TMEM is freed
+      mma_commit(&sm.drain);
+      int never = 0;
+      mbar_wait(&sm.drain, 0, &never);
     }
   } else {
     // epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 = tile rows
     const int quad = warp & 3;
-    const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sm.acc_full, 0, abort)) && !*abort;
-    if (ok) {
+    float* stage = sm.out[warp - 2];
+    int i = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
+      const int buf = i & 1;
+      const bool ok = __all_sync(kFull, mbar_wait(&sm.acc_full[buf], (i >> 1) & 1, abort));
+      if (!ok || *abort) {
+        if (lane == 0 && !*abort) fail_status(a.status, &sm.abort, kDevErrTimeoutMma);
+        break;
+      }
       tc_fence_after_sync();
-      float* stage = &sm.a[0][0][0] + size_t(warp - 2) * 32 * kLtStagePitch;
-      const uint32_t t_row = tmem + (uint32_t(quad * 32) << 16);
+      const LtTile tl = lt_tile(t, nrt, nct);
+      const uint32_t t_row = tmem + (uint32_t(quad * 32) << 16) + uint32_t(buf * kLtN);
+      const int row0 = tl.r0 + quad * 32;  // this warp's first tile row
+      float* out = a.logits + (size_t(tl.bh) * g.nb + row0) * ld + tl.c0;
 #pragma unroll 1
       for (int cc = 0; cc < kLtN / 32; ++cc) {
         uint32_t v[32];
         tmem_ld32(t_row + 32 * cc, v);
         tmem_wait_ld();
-        float4* dst = reinterpret_cast<float4*>(stage + lane * kLtStagePitch + 32 * cc);
+        float4* dst = reinterpret_cast<float4*>(stage + lane * kLtStagePitch);
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          dst[i] = make_float4(__uint_as_float(v[4 * i]) * a.scale,
-                               __uint_as_float(v[4 * i + 1]) * a.scale,
-                               __uint_as_float(v[4 * i + 2]) * a.scale,
-                               __uint_as_float(v[4 * i + 3]) * a.scale);
+        for (int k = 0; k < 8; ++k)
+          dst[k] = make_float4(__uint_as_float(v[4 * k]) * a.scale,
+                               __uint_as_float(v[4 * k + 1]) * a.scale,
+                               __uint_as_float(v[4 * k + 2]) * a.scale,
+                               __uint_as_float(v[4 * k + 3]) * a.scale);
+        __syncwarp();
+        // four whole 128-byte row segments per store instruction
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int rr = 4 * k + (lane >> 3), c4 = lane & 7;
+          if (row0 + rr < g.nb)
+            reinterpret_cast<float4*>(out + size_t(rr) * ld + 32 * cc)[c4] =
+                reinterpret_cast<const float4*>(stage + rr * kLtStagePitch)[c4];
+        }
+        __syncwarp();
       }
+      tc_fence_before_sync();
       __syncwarp();
-      // row by row: the warp writes 1 KB contiguous per row
-      for (int rr = 0; rr < 32; ++rr) {
-        const int row = r0 + quad * 32 + rr;
-        if (row >= g.nb) break;  // rows ascend with rr
-        const float* src = stage + rr * kLtStagePitch;
-        float* out = a.logits + (size_t(row_base) + row) * ld + c0;
-        reinterpret_cast<float4*>(out)[lane] = reinterpret_cast<const float4*>(src)[lane];
-        reinterpret_cast<float4*>(out + 128)[lane] = reinterpret_cast<const float4*>(src + 128)[lane];
-      }
+      if (lane == 0) mbar_arrive(&sm.acc_empty[buf]);
     }
   }
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
-  if (warp == 1) tmem_dealloc(tmem, 256);
+  if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
 // ------------------------------------------------------------------ select
@@ -198,11 +231,13 @@ constexpr int kSelWarps = 8;
 constexpr int kCandCap = 256;      // compacted search window per warp (8 per lane)
 constexpr int kMaxRowWords = 192;  // keep-bitmap words of a row (nb <= 6144)
 constexpr int kRegVPL = 96;        // longest row held in registers (nb <= 3072)
+constexpr int kLaneCap = 16;       // window masses a lane appends to its own column
 // Per-warp shared work area, used in turn by the leading-bit histogram
-// (32 buckets x 32 lanes), the compacted window (words 0..255) and the keep
-// bitmap (words 256..447).
+// (32 buckets x 32 lanes, words 0..1023), then the lanes' window columns
+// (words 0..511), the packed window (512..767) and the keep bitmap (768..959).
 constexpr int kSelWork = 32 * 32;
-constexpr int kRbitsAt = kCandCap;
+constexpr int kDenseAt = kLaneCap * 32;
+constexpr int kRbitsAt = kDenseAt + kCandCap;
 static_assert(kRbitsAt + kMaxRowWords <= kSelWork, "select work area");
 
 // A row's integer masses, VPL per lane (column j in lane j % 32, slot
@@ -241,6 +276,33 @@ __device__ __forceinline__ uint32_t mass_at_least(const Store& m, uint32_t c) {
 #pragma unroll
     for (int i = 0; i + w < kAcc; i += 2 * w) acc[i] += acc[i + w];
   return __reduce_add_sync(kFull, acc[0]);
+}
+
+// The bits of tau below its leading bit e, one by one, over the packed
+// window (wcnt masses in [2^e, 2^(e+1)), N per lane); `above` is the mass
+// above the window. Also counts the masses equal to tau.
+template <int N>
+__device__ __forceinline__ void window_search(const uint32_t* dense, int wcnt, int lane, int e,
+                                              uint32_t above, uint32_t tgt, uint32_t& tau,
+                                              uint32_t& keep_ties, uint32_t& n_tau) {
+  RowStore<N, false> cwr;
+#pragma unroll
+  for (int k = 0; k < N; ++k) {
+    const int at = 32 * k + lane;
+    cwr.set(k, at < wcnt ? dense[at] : 0u);  // 0 is below every candidate
+  }
+  uint32_t x = 1u << e;
+#pragma unroll 1
+  for (int b = e - 1; b >= 0; --b) {
+    const uint32_t t = x | (1u << b);
+    if (above + mass_at_least<N>(cwr, t) >= tgt) x = t;
+  }
+  tau = x;
+  uint32_t eq = 0;
+#pragma unroll
+  for (int k = 0; k < N; ++k) eq += cwr.get(k) == tau ? 1u : 0u;
+  n_tau = __reduce_add_sync(kFull, eq);
+  keep_ties = (tgt - above - mass_at_least<N>(cwr, tau + 1) + tau - 1) / tau;
 }
 
 // VPL = values per lane: column j of the row sits in lane j % 32, slot j / 32.
@@ -299,8 +361,9 @@ __global__ void __launch_bounds__(kSelWarps * 32, VPL <= 32 ? 4 : (VPL <= 64 ? 2
   //     then sums row b, and a suffix scan over the lanes gives G(2^b) in
   //     lane b): e is the highest b with G(2^b) >= target, and G(2^(e+1)),
   //     the mass above the window [2^e, 2^(e+1)), comes with it.
-  //  2. The window's masses are compacted to shared memory (if at most 256)
-  //     and the lower bits of tau found one by one over them alone, the mass
+  //  2. The window's masses are compacted to shared memory (if at most 256,
+  //     and at most 16 in any lane) and the lower bits of tau found one by
+  //     one over them alone (1, 2, 4 or 8 per lane), the mass
   //     above the window entering as a constant; a longer window is searched
   //     bit by bit over the whole row.
   // Blocks with mass > tau are kept, and of those with mass == tau the first
@@ -340,35 +403,26 @@ __global__ void __launch_bounds__(kSelWarps * 32, VPL <= 32 ? 4 : (VPL <= 64 ? 2
       const int e = 31 - __clz(__ballot_sync(kFull, gs >= tgt));
       const uint32_t above = __shfl_sync(kFull, gs, e + 1);
       uint32_t x = 1u << e;
-      int wcnt = 0;  // compact the window [x, 2x); order does not matter for sums
+      // compact the window [x, 2x): each lane appends its window masses to
+      // its own column, then the columns are packed (order does not matter
+      // for sums)
+      int wcnt = 0;
+      uint32_t* dense = work + kDenseAt;
 #pragma unroll
       for (int i = 0; i < VPL; ++i) {
         const uint32_t mi = m.get(i);
         const bool in = (mi - x) < x;  // unsigned: x <= m < 2x
         const unsigned bal = __ballot_sync(kFull, in);
         const int at = wcnt + __popc(bal & lanemask_lt());
-        if (in && at < kCandCap) work[at] = mi;
+        if (in && at < kCandCap) dense[at] = mi;
         wcnt += __popc(bal);
       }
       __syncwarp();
       if (wcnt <= kCandCap) {
-        RowStore<kCandCap / 32, false> cwr;
-#pragma unroll
-        for (int k = 0; k < kCandCap / 32; ++k) {
-          const int at = 32 * k + lane;
-          cwr.set(k, at < wcnt ? work[at] : 0u);  // 0 is below every candidate
-        }
-#pragma unroll 1
-        for (int b = e - 1; b >= 0; --b) {
-          const uint32_t t = x | (1u << b);
-          if (above + mass_at_least<kCandCap / 32>(cwr, t) >= tgt) x = t;
-        }
-        tau = x;
-        uint32_t eq = 0;
-#pragma unroll
-        for (int k = 0; k < kCandCap / 32; ++k) eq += cwr.get(k) == tau ? 1u : 0u;
-        n_tau = __reduce_add_sync(kFull, eq);
-        keep_ties = (tgt - above - mass_at_least<kCandCap / 32>(cwr, tau + 1) + tau - 1) / tau;
+        if (wcnt <= 32) window_search<1>(dense, wcnt, lane, e, above, tgt, tau, keep_ties, n_tau);
+        else if (wcnt <= 64) window_search<2>(dense, wcnt, lane, e, above, tgt, tau, keep_ties, n_tau);
+        else if (wcnt <= 128) window_search<4>(dense, wcnt, lane, e, above, tgt, tau, keep_ties, n_tau);
+        else window_search<8>(dense, wcnt, lane, e, above, tgt, tau, keep_ties, n_tau);
       } else {
 #pragma unroll 1
         for (int b = e - 1; b >= 0; --b) {
@@ -576,7 +630,12 @@ cudaError_t launch_logits(const MaskArgs& a, const Geometry& g, int ld, cudaStre
   cudaError_t e = cudaFuncSetAttribute(logits_tc_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const dim3 grid(unsigned(ld / kLtN), unsigned((g.nb + kLtM - 1) / kLtM), unsigned(g.BH));
+  int dev = 0, nsm = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  const long ntiles = long(g.BH) * ((g.nb + kLtM - 1) / kLtM) * (ld / kLtN);
+  const unsigned grid = unsigned(ntiles < nsm ? ntiles : nsm);  // one CTA per SM
   logits_tc_kernel<D><<<grid, kLtThreads, smem, stream>>>(a, g, ld);
   return cudaGetLastError();
 }
