@@ -231,12 +231,11 @@ constexpr int kSelWarps = 8;
 constexpr int kCandCap = 256;      // compacted search window per warp (8 per lane)
 constexpr int kMaxRowWords = 192;  // keep-bitmap words of a row (nb <= 6144)
 constexpr int kRegVPL = 96;        // longest row held in registers (nb <= 3072)
-constexpr int kLaneCap = 16;       // window masses a lane appends to its own column
 // Per-warp shared work area, used in turn by the leading-bit histogram
-// (32 buckets x 32 lanes, words 0..1023), then the lanes' window columns
-// (words 0..511), the packed window (512..767) and the keep bitmap (768..959).
+// (32 buckets x 32 lanes, words 0..1023), then the packed window (words
+// 0..255) and the keep bitmap (256..447).
 constexpr int kSelWork = 32 * 32;
-constexpr int kDenseAt = kLaneCap * 32;
+constexpr int kDenseAt = 0;
 constexpr int kRbitsAt = kDenseAt + kCandCap;
 static_assert(kRbitsAt + kMaxRowWords <= kSelWork, "select work area");
 
@@ -361,9 +360,9 @@ __global__ void __launch_bounds__(kSelWarps * 32, VPL <= 32 ? 4 : (VPL <= 64 ? 2
   //     then sums row b, and a suffix scan over the lanes gives G(2^b) in
   //     lane b): e is the highest b with G(2^b) >= target, and G(2^(e+1)),
   //     the mass above the window [2^e, 2^(e+1)), comes with it.
-  //  2. The window's masses are compacted to shared memory (if at most 256,
-  //     and at most 16 in any lane) and the lower bits of tau found one by
-  //     one over them alone (1, 2, 4 or 8 per lane), the mass
+  //  2. The window's masses are compacted to shared memory (if at most 256)
+  //     and the lower bits of tau found one by one over them alone (1, 2, 4
+  //     or 8 per lane), the mass
   //     above the window entering as a constant; a longer window is searched
   //     bit by bit over the whole row.
   // Blocks with mass > tau are kept, and of those with mass == tau the first
@@ -403,9 +402,7 @@ __global__ void __launch_bounds__(kSelWarps * 32, VPL <= 32 ? 4 : (VPL <= 64 ? 2
       const int e = 31 - __clz(__ballot_sync(kFull, gs >= tgt));
       const uint32_t above = __shfl_sync(kFull, gs, e + 1);
       uint32_t x = 1u << e;
-      // compact the window [x, 2x): each lane appends its window masses to
-      // its own column, then the columns are packed (order does not matter
-      // for sums)
+      // compact the window [x, 2x); order does not matter for sums
       int wcnt = 0;
       uint32_t* dense = work + kDenseAt;
 #pragma unroll
