@@ -3,15 +3,16 @@
 //
 //  logits_tc_kernel  L[bh][r][j] = Qbar[r] . Kbar[j] / sqrt(d) for every pair
 //                 of blocks of a head on the TF32 tensor cores (three products
-//                 of a hi / lo split: fp32-level accuracy), 128 x 256 output
-//                 tiles, stored in the workspace;
+//                 of a hi / lo split: fp32-level accuracy), a persistent
+//                 kernel over 128 x 256 output tiles, stored in the workspace;
 //  select_kernel  one warp per q-block row, the row held in registers:
 //                 softmax, then the CDF threshold without sorting. k-block j
 //                 is kept iff the probability mass ranked before it (descending
 //                 order, ties by index) is < 1 - thr. With masses in 2^-30
 //                 fixed point (integer sums, so the result is bit-identical
-//                 run to run), a bitwise binary search over warp-reduced
-//                 partial sums finds the mass tau of the last kept block; of
+//                 run to run), a leading-bit histogram and a bitwise search
+//                 over the compacted octave find the mass tau of the last
+//                 kept block; of
 //                 the blocks whose mass equals tau, those that keep the
 //                 running mass below the threshold are kept in ascending index
 //                 order. Then the OR with the static STA window, the ascending
