@@ -547,24 +547,43 @@ __global__ void __launch_bounds__(kUnionMaxWarps * 32) union_kernel(MaskArgs a, 
     const int nbits = pf - 32 * w;
     return nbits < 32 ? x & ((1u << nbits) - 1u) : x;
   };
-  // Greedy pairing along time, 32 patches per lane-word at once: a block
-  // present in frame t whose frame t - 1 block is present and not already the
-  // second of a pair becomes the second of a pair.
-  for (int w = lane; w < fw; w += 32) {
-    uint32_t prev_in = 0u, prev_pair = 0u;
-    for (int t = 0; t < g.nt; ++t) {
-      const uint32_t in = frame_word(t, w);
-      const uint32_t pair = prev_in & ~prev_pair & in;
-      if (t > 0) {
-        firstF[(t - 1) * fw + w] = pair;
-        leftF[(t - 1) * fw + w] = prev_in & ~prev_pair & ~pair;
+  // Greedy pairing along time: a block present in frame t whose frame t - 1
+  // block is present and not already the second of a pair becomes the second
+  // of a pair. Per bit, pair_t = a_t & ~pair_(t-1) with a_t = in_(t-1) & in_t:
+  // each frame applies x -> (x & k) ^ v to the previous frame's pair bits
+  // (k = v = a_t), and these maps compose associatively, so the pair bits of
+  // 32 frames come from one scan over the lanes (lane = frame), 32 patches
+  // per word at once. firstF[t] marks the first blocks of the pairs (t, t+1)
+  // (= pair_(t+1)); leftF first holds in_t, then keeps the unpaired blocks.
+  for (int w = 0; w < fw; ++w) {
+    uint32_t carry_in = 0u, carry_pair = 0u;  // frame 32 c - 1: presence, pair bits
+    for (int t0 = 0; t0 < g.nt; t0 += 32) {
+      const int t = t0 + lane;
+      const uint32_t in = t < g.nt ? frame_word(t, w) : 0u;
+      uint32_t prev = __shfl_up_sync(kFull, in, 1);
+      if (lane == 0) prev = carry_in;
+      uint32_t k = prev & in, v = k;  // a_t
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t ke = __shfl_up_sync(kFull, k, o), ve = __shfl_up_sync(kFull, v, o);
+        if (lane >= o) {  // this map after the earlier composite
+          v = (ve & k) ^ v;
+          k = ke & k;
+        }
       }
-      prev_in = in;
-      prev_pair = pair;
+      const uint32_t pair = (carry_pair & k) ^ v;
+      if (t < g.nt) {
+        if (t > 0) firstF[(t - 1) * fw + w] = pair;
+        leftF[t * fw + w] = in;
+      }
+      carry_in = __shfl_sync(kFull, in, 31);
+      carry_pair = __shfl_sync(kFull, pair, 31);
     }
-    firstF[(g.nt - 1) * fw + w] = 0u;
-    leftF[(g.nt - 1) * fw + w] = prev_in & ~prev_pair;
+    if (lane == 0) firstF[(g.nt - 1) * fw + w] = 0u;
   }
+  __syncwarp();
+  for (int i = lane; i < nf; i += 32)  // unpaired: in_t & ~pair_t & ~pair_(t+1)
+    leftF[i] &= ~firstF[i] & (i >= fw ? ~firstF[i - fw] : ~0u);
   __syncwarp();
 
   // Emission in ascending block order (frame-major words are in block
