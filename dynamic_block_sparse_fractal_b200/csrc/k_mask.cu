@@ -279,17 +279,20 @@ __device__ __forceinline__ uint32_t mass_at_least(const Store& m, uint32_t c) {
 }
 
 // The bits of tau below its leading bit e, one by one, over the packed
-// window (wcnt masses in [2^e, 2^(e+1)), N per lane); `above` is the mass
-// above the window. Also counts the masses equal to tau.
+// window (wcnt masses in [2^e, 2^(e+1)), N per lane: the first n0 in d0, the
+// rest in d1); `above` is the mass above the window. Also counts the masses
+// equal to tau.
 template <int N>
-__device__ __forceinline__ void window_search(const uint32_t* dense, int wcnt, int lane, int e,
-                                              uint32_t above, uint32_t tgt, uint32_t& tau,
-                                              uint32_t& keep_ties, uint32_t& n_tau) {
+__device__ __forceinline__ void window_search(const uint32_t* d0, int n0, const uint32_t* d1,
+                                              int wcnt, int lane, int e, uint32_t above,
+                                              uint32_t tgt, uint32_t& tau, uint32_t& keep_ties,
+                                              uint32_t& n_tau) {
   RowStore<N, false> cwr;
 #pragma unroll
   for (int k = 0; k < N; ++k) {
     const int at = 32 * k + lane;
-    cwr.set(k, at < wcnt ? dense[at] : 0u);  // 0 is below every candidate
+    // 0 is below every candidate
+    cwr.set(k, at < n0 ? d0[at] : (at < wcnt ? d1[at - n0] : 0u));
   }
   uint32_t x = 1u << e;
 #pragma unroll 1
@@ -417,10 +420,14 @@ __global__ void __launch_bounds__(kSelWarps * 32, VPL <= 32 ? 4 : (VPL <= 64 ? 2
       }
       __syncwarp();
       if (wcnt <= kCandCap) {
-        if (wcnt <= 32) window_search<1>(dense, wcnt, lane, e, above, tgt, tau, keep_ties, n_tau);
-        else if (wcnt <= 64) window_search<2>(dense, wcnt, lane, e, above, tgt, tau, keep_ties, n_tau);
-        else if (wcnt <= 128) window_search<4>(dense, wcnt, lane, e, above, tgt, tau, keep_ties, n_tau);
-        else window_search<8>(dense, wcnt, lane, e, above, tgt, tau, keep_ties, n_tau);
+        if (wcnt <= 32)
+          window_search<1>(dense, wcnt, dense, wcnt, lane, e, above, tgt, tau, keep_ties, n_tau);
+        else if (wcnt <= 64)
+          window_search<2>(dense, wcnt, dense, wcnt, lane, e, above, tgt, tau, keep_ties, n_tau);
+        else if (wcnt <= 128)
+          window_search<4>(dense, wcnt, dense, wcnt, lane, e, above, tgt, tau, keep_ties, n_tau);
+        else
+          window_search<8>(dense, wcnt, dense, wcnt, lane, e, above, tgt, tau, keep_ties, n_tau);
       } else {
 #pragma unroll 1
         for (int b = e - 1; b >= 0; --b) {
@@ -503,6 +510,246 @@ __global__ void __launch_bounds__(kSelWarps * 32, VPL <= 32 ? 4 : (VPL <= 64 ? 2
     pos += __shfl_sync(kFull, inc, 31);
   }
   if (lane == 0) a.cnt[row] = pos;
+}
+
+// ------------------------------------------------------------------ select, two warps per row
+// Rows of 1025..2048 blocks: a pair of warps per row, 32 masses per lane each
+// (warp h holds columns 1024 h + lane + 32 i), so that twice as many rows are
+// in flight per SM as with one warp holding 64 masses per lane (registers
+// bound the occupancy). The operations are those of select_kernel in the same
+// order: the row sum continues warp 0's per-lane partial sums in warp 1, and
+// integer sums are exact, so the kept sets are identical. The two warps meet
+// at a named barrier of their own.
+constexpr int kPairs = 4;      // rows per CTA
+constexpr int kPairHV = 32;    // masses per lane and warp
+constexpr int kPairRbitsAt = 2 * kCandCap;  // bitmap after the two window halves
+static_assert(kPairRbitsAt + 64 <= kSelWork, "pair work area");
+
+__global__ void __launch_bounds__(kPairs * 64, 4)
+    select_pair_kernel(const float* __restrict__ L, MaskArgs a, Geometry g, int ld) {
+  __shared__ __align__(16) uint32_t work_all[kPairs][kSelWork];
+  __shared__ uint32_t xch_all[kPairs][64];  // per pair: values passed between the warps
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pr = warp >> 1, h = warp & 1;
+  const long row = long(blockIdx.x) * kPairs + pr;
+  if (row >= long(g.BH) * g.nb) return;  // both warps of the pair
+  const uint32_t bar_id = 1u + uint32_t(pr);
+  const int nb = g.nb;
+  const int qb = int(row % nb);
+  const float* Lr = L + size_t(row) * ld;
+  uint32_t* work = work_all[pr];
+  uint32_t* xch = xch_all[pr];  // [0..2]: maxima, sum; [8..39]: partial sums; [48..]: integers
+  float* xf = reinterpret_cast<float*>(xch);
+  const int j0 = h * 32 * kPairHV;
+  constexpr float kLog2e = 1.4426950408889634f;
+
+  // ---- row softmax to integer masses m = p * 2^30
+  RowStore<kPairHV, false> m;
+  {
+    float mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < kPairHV; ++i) {
+      const int j = j0 + lane + 32 * i;
+      const float v = j < nb ? __ldg(Lr + j) : -INFINITY;
+      m.set(i, __float_as_uint(v));
+      mx = fmaxf(mx, v);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+    if (lane == 0) xf[h] = mx;
+    named_barrier_sync(bar_id, 64);
+    mx = fmaxf(xf[0], xf[1]);
+    const float shift = -mx * kLog2e;
+#pragma unroll
+    for (int i = 0; i < kPairHV; ++i)  // exactly 0 in the padding slots
+      m.set(i, __float_as_uint(ex2_approx(fmaf(__uint_as_float(m.get(i)), kLog2e, shift))));
+    if (h == 0) {
+      float sum = 0.f;
+#pragma unroll
+      for (int i = 0; i < kPairHV; ++i) sum += __uint_as_float(m.get(i));
+      xf[8 + lane] = sum;
+    }
+    named_barrier_sync(bar_id, 64);
+    if (h == 1) {
+      float sum = xf[8 + lane];
+#pragma unroll
+      for (int i = 0; i < kPairHV; ++i) sum += __uint_as_float(m.get(i));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(kFull, sum, o);
+      if (lane == 0) xf[2] = sum;
+    }
+    named_barrier_sync(bar_id, 64);
+    const float to_fx = 1073741824.0f / xf[2];  // 2^30 / sum
+#pragma unroll
+    for (int i = 0; i < kPairHV; ++i) m.set(i, __float2uint_rn(__uint_as_float(m.get(i)) * to_fx));
+  }
+
+  // ---- CDF threshold, as in select_kernel: the leading-bit histogram (one
+  // table for the pair), the window compacted by each warp into its own half,
+  // searched by warp 0
+  bool keep_all = a.dense != 0;
+  uint32_t tau = 0, keep_ties = 0, n_tau = 0;
+  if (!keep_all) {
+    const uint32_t tgt = a.target_fx;
+    uint4* work4 = reinterpret_cast<uint4*>(work);
+#pragma unroll
+    for (int k = h * 32 + lane; k < kSelWork / 4; k += 64) work4[k] = make_uint4(0u, 0u, 0u, 0u);
+    named_barrier_sync(bar_id, 64);
+#pragma unroll
+    for (int i = 0; i < kPairHV; ++i) {
+      const uint32_t mi = m.get(i);
+      if (mi != 0u) atomicAdd(work + (31 - __clz(mi)) * 32 + lane, mi);
+    }
+    named_barrier_sync(bar_id, 64);
+    uint32_t gs = 0;
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      const uint4 q = work4[lane * 8 + ((lane + s) & 7)];
+      gs += (q.x + q.y) + (q.z + q.w);
+    }
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_down_sync(kFull, gs, o);
+      if (lane + o < 32) gs += t;
+    }
+    const uint32_t total = __shfl_sync(kFull, gs, 0);
+    named_barrier_sync(bar_id, 64);  // both warps have read the table
+    if (total < tgt) {
+      keep_all = true;
+    } else {
+      const int e = 31 - __clz(__ballot_sync(kFull, gs >= tgt));
+      const uint32_t above = __shfl_sync(kFull, gs, e + 1);
+      uint32_t x = 1u << e;
+      uint32_t* half = work + h * kCandCap;
+      int wc = 0;
+#pragma unroll
+      for (int i = 0; i < kPairHV; ++i) {
+        const uint32_t mi = m.get(i);
+        const bool in = (mi - x) < x;  // unsigned: x <= m < 2x
+        const unsigned bal = __ballot_sync(kFull, in);
+        const int at = wc + __popc(bal & lanemask_lt());
+        if (in && at < kCandCap) half[at] = mi;
+        wc += __popc(bal);
+      }
+      if (lane == 0) xch[48 + h] = uint32_t(wc);
+      named_barrier_sync(bar_id, 64);
+      const int wc0 = int(xch[48]), wcnt = wc0 + int(xch[49]);
+      if (wcnt <= kCandCap) {
+        if (h == 0) {
+          const uint32_t* d1 = work + kCandCap;
+          if (wcnt <= 32)
+            window_search<1>(work, wc0, d1, wcnt, lane, e, above, tgt, tau, keep_ties, n_tau);
+          else if (wcnt <= 64)
+            window_search<2>(work, wc0, d1, wcnt, lane, e, above, tgt, tau, keep_ties, n_tau);
+          else if (wcnt <= 128)
+            window_search<4>(work, wc0, d1, wcnt, lane, e, above, tgt, tau, keep_ties, n_tau);
+          else
+            window_search<8>(work, wc0, d1, wcnt, lane, e, above, tgt, tau, keep_ties, n_tau);
+          if (lane == 0) {
+            xch[50] = tau;
+            xch[51] = keep_ties;
+            xch[52] = n_tau;
+          }
+        }
+        named_barrier_sync(bar_id, 64);
+        tau = xch[50];
+        keep_ties = xch[51];
+        n_tau = xch[52];
+      } else {  // a long window: bit by bit over both warps' masses
+#pragma unroll 1
+        for (int b = e - 1; b >= 0; --b) {
+          const uint32_t t = x | (1u << b);
+          const uint32_t part = mass_at_least<kPairHV>(m, t);
+          uint32_t* slot = xch + 56 + 2 * (b & 1);  // alternate slots: no overwrite before read
+          if (lane == 0) slot[h] = part;
+          named_barrier_sync(bar_id, 64);
+          if (slot[0] + slot[1] >= tgt) x = t;
+        }
+        tau = x;
+        const uint32_t part = mass_at_least<kPairHV>(m, tau + 1);
+        if (lane == 0) xch[60 + h] = part;
+        named_barrier_sync(bar_id, 64);
+        keep_ties = (tgt - (xch[60] + xch[61]) + tau - 1) / tau;
+      }
+    }
+  }
+
+  // ---- keep bitmap: warp h writes words 32 h .. 32 h + 31; ties in index
+  // order (warp 0's columns first) unless every mass equal to tau is kept
+  uint32_t* rbits = work + kPairRbitsAt;
+  if (keep_all || n_tau == keep_ties) {
+#pragma unroll
+    for (int i = 0; i < kPairHV; ++i) {
+      if (j0 + 32 * i < nb) {  // warp-uniform
+        const bool nab = keep_all ? j0 + lane + 32 * i < nb : m.get(i) >= tau;
+        const unsigned kb = __ballot_sync(kFull, nab);
+        if (lane == 0) rbits[h * kPairHV + i] = kb;
+      }
+    }
+  } else {
+    uint32_t ties = 0;
+    if (h == 1) named_barrier_sync(bar_id, 64);  // warp 0's tie count first
+    if (h == 1) ties = xch[62];
+#pragma unroll
+    for (int i = 0; i < kPairHV; ++i) {
+      if (j0 + 32 * i < nb) {  // warp-uniform
+        const uint32_t mi = m.get(i);
+        bool nab = mi > tau;
+        const bool tie = mi == tau;
+        const unsigned tb = __ballot_sync(kFull, tie);
+        if (tie) nab = (ties + __popc(tb & lanemask_lt())) < keep_ties;
+        ties += __popc(tb);
+        const unsigned kb = __ballot_sync(kFull, nab);
+        if (lane == 0) rbits[h * kPairHV + i] = kb;
+      }
+    }
+    if (h == 0) {
+      if (lane == 0) xch[62] = ties;
+      named_barrier_sync(bar_id, 64);
+    }
+  }
+  named_barrier_sync(bar_id, 64);  // the bitmap is complete
+  if (a.sta_t >= 0) {
+    int tq, hq, wq;
+    block_coords(g, qb, tq, hq, wq);
+    const int t0 = max(tq - a.sta_t, 0), t1 = min(tq + a.sta_t, g.nt - 1);
+    const int h0 = max(hq - a.sta_h, 0), h1 = min(hq + a.sta_h, g.nh - 1);
+    const int w0 = max(wq - a.sta_w, 0), w1 = min(wq + a.sta_w, g.nw - 1);
+    const int nw_ = w1 - w0 + 1, nhw = (h1 - h0 + 1) * nw_;
+    const int cells = (t1 - t0 + 1) * nhw;
+    for (int cidx = h * 32 + lane; cidx < cells; cidx += 64) {
+      const int ct = cidx / nhw, r = cidx - ct * nhw, ch = r / nw_, cw = r - ch * nw_;
+      const int j = ((t0 + ct) * g.nh + h0 + ch) * g.nw + w0 + cw;
+      atomicOr(&rbits[j >> 5], 1u << (j & 31));
+    }
+    named_barrier_sync(bar_id, 64);
+  }
+
+  // ---- ascending kept list, bitmap and count: warp h takes words 32 h ..
+  const int nwords = bitmap_words(g);
+  uint32_t* bits = a.bits + size_t(row) * nwords;
+  int32_t* out_idx = a.idx + size_t(row) * nb;
+  int pos = 0;
+  if (h == 1) pos = int(__reduce_add_sync(kFull, uint32_t(__popc(rbits[lane]))));
+  {
+    const int wi = 32 * h + lane;
+    uint32_t w = wi < nwords ? rbits[wi] : 0u;
+    if (wi < nwords) bits[wi] = w;
+    const int cnt = __popc(w);
+    int inc = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(kFull, inc, o);
+      if (lane >= o) inc += t;
+    }
+    int o = pos + inc - cnt;
+    while (w) {
+      out_idx[o++] = 32 * wi + __ffs(w) - 1;
+      w &= w - 1u;
+    }
+    pos += __shfl_sync(kFull, inc, 31);
+  }
+  if (h == 1 && lane == 0) a.cnt[row] = pos;
 }
 
 // ------------------------------------------------------------------ union
@@ -641,6 +888,13 @@ cudaError_t launch_select(const MaskArgs& a, const Geometry& g, int ld, cudaStre
   return cudaGetLastError();
 }
 
+cudaError_t launch_select_pair(const MaskArgs& a, const Geometry& g, int ld, cudaStream_t stream) {
+  const long rows = long(g.BH) * g.nb;
+  select_pair_kernel<<<unsigned((rows + kPairs - 1) / kPairs), kPairs * 64, 0, stream>>>(
+      a.logits, a, g, ld);
+  return cudaGetLastError();
+}
+
 template <int D>
 cudaError_t launch_logits(const MaskArgs& a, const Geometry& g, int ld, cudaStream_t stream) {
   const int smem = int(sizeof(LogitsSmem) + 1024);
@@ -671,7 +925,7 @@ cudaError_t launch_mask(const MaskArgs& a, const Geometry& g, cudaStream_t strea
   else if (vpl <= 8) e = launch_select<8>(a, g, ld, stream);
   else if (vpl <= 16) e = launch_select<16>(a, g, ld, stream);
   else if (vpl <= 32) e = launch_select<32>(a, g, ld, stream);
-  else if (vpl <= 64) e = launch_select<64>(a, g, ld, stream);
+  else if (vpl <= 64) e = launch_select_pair(a, g, ld, stream);
   else if (vpl <= 96) e = launch_select<96>(a, g, ld, stream);
   else e = launch_select<192>(a, g, ld, stream);
   if (e != cudaSuccess) return e;
