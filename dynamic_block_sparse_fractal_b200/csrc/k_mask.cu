@@ -16,7 +16,9 @@
 //                 the blocks whose mass equals tau, those that keep the
 //                 running mass below the threshold are kept in ascending index
 //                 order. Then the OR with the static STA window, the ascending
-//                 kept list and the row's keep bitmap;
+//                 kept list and the row's keep bitmap (select_pair_kernel:
+//                 the same with two warps per row, for rows of 1025..2048
+//                 blocks);
 //  union_kernel   one warp per query tile (two q-blocks): the union of the
 //                 two bitmaps as a list of k-blocks tagged with which q-block
 //                 keeps each, first the steps that pair one patch in frames t
