@@ -303,6 +303,7 @@ def run_ours(args, w, rank, world):
                                                              stream)
     backward = None if args.no_backward else measure_backward(api, desc, w, q, k, v, ws,
                                                               kept_pairs, dev, stream)
+    radius = None if args.no_radius else measure_radius(api, desc, w, q, k, dev, stream)
 
     peaks, src = load_peaks()
     ms_step = total_ms / args.steps
@@ -356,6 +357,9 @@ def run_ours(args, w, rank, world):
     if backward is not None:
         backward["frac"] = round(backward["kept_tflops"] / peak, 4)
         line["backward"] = backward
+    if radius is not None:
+        radius["entropy_frac"] = round(radius["entropy_tensor_tflops"] / peak, 4)
+        line["radius_mask"] = radius
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -442,6 +446,43 @@ def measure_heatmap(api, desc, w, q, k, ws, views, dev, stream, reps=3):
             "note": "one dense Q K^T pass (row log-sum-exp + raw block maxima, then per-row "
                     "reduction of the maxima); time includes zeroing the map",
             "mask_recall": round(recall, 4)}
+
+
+def measure_radius(api, desc, w, q, k, dev, stream, tau=2.0, gamma=0.25, vote_min=1, reps=5):
+    """Times the Token Radius Attention mask builder outside the step, in a
+    workspace of its own: the per-token entropy pass (one dense Q K^T) and the
+    radius plan (block votes, lists, tile unions, tile order) for one setting
+    of the key budget tau, the temporal decay gamma and the vote threshold, and
+    reports the density of the mask it builds."""
+    import torch
+    ws_r = api.alloc_workspace(desc)
+    ent = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    api.token_entropy(desc, q, k, ws_r, ent)
+    api.plan_radius(desc, tau, gamma, vote_min, ent, ws_r)
+    e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    api.token_entropy(desc, q, k, ws_r, ent)
+    e1.record(stream)
+    for _ in range(reps):
+        api.plan_radius(desc, tau, gamma, vote_min, ent, ws_r)
+    e2.record(stream)
+    torch.cuda.synchronize(dev)
+    ent_ms = e0.elapsed_time(e1)
+    plan_us = e1.elapsed_time(e2) / reps * 1e3
+    st = api.check(desc, ws_r)
+    if st != api.SA_OK:
+        raise SystemExit(f"device status after the radius mask: {api.status_string(st)}")
+    cnt = api.get_mask(desc, ws_r)["cnt"]
+    density = float(cnt.double().sum().item()) / (w.BH * w.nb * w.nb)
+    qk_flops = 2.0 * w.S * w.S * w.d * w.BH  # one dense Q K^T
+    return {"tau": tau, "gamma": gamma, "vote_min": vote_min,
+            "entropy_ms": round(ent_ms, 3),
+            "entropy_tensor_tflops": round(qk_flops / (ent_ms * 1e-3) / 1e12, 2),
+            "plan_us": round(plan_us, 1), "density": round(density, 4),
+            "mean_entropy_nats": round(float(ent.double().mean().item()), 4),
+            "note": "entropy pass = the map kernel in entropy mode; plan = votes, lists, "
+                    "tile unions and order"}
 
 
 def measure_backward(api, desc, w, q, k, v, ws, kept_pairs, dev, stream, reps=3):
@@ -546,6 +587,8 @@ def main():
                     help="skip the block max-pooled attention map measurement")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the gradient (backward) measurement")
+    ap.add_argument("--no-radius", action="store_true",
+                    help="skip the radius (TRA) mask measurement")
     ap.add_argument("--heads", type=int, default=None,
                     help="run the workload's grid with this many heads (small ncu captures); "
                          "the line's config then names the changed workload")
