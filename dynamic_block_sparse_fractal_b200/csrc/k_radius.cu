@@ -21,8 +21,11 @@
 // pruned first when even the q-block's bounding box, at the largest radius of
 // its queries, misses it.
 //
-// One warp per q-block row; eight rows per CTA. The per-frame tables f and
-// 1 / (pi Z) are built once per CTA in fp64 and kept as fp32.
+// One warp per q-block row; eight rows per CTA. Each lane holds two of the
+// q-block's 64 queries; the k-blocks are taken 32 at a time (lane = k-block)
+// for the pruning test, then the warp walks the unpruned ones and its lanes
+// vote for each at once. The per-frame tables f and 1 / (pi Z) are built once
+// per CTA in fp64 and kept as fp32.
 #include <cuda_runtime.h>
 
 #include "kernels.cuh"
@@ -42,8 +45,6 @@ __device__ __forceinline__ int dist_to_range(int x, int lo, int hi) {
 __global__ void __launch_bounds__(kRadWarps * 32) radius_kernel(RadiusArgs a, Geometry g) {
   __shared__ float f_tab[kRadMaxFrames];     // exp(-2 gamma delta)
   __shared__ float zinv_tab[kRadMaxFrames];  // 1 / (pi Z(t))
-  __shared__ float r2_all[kRadWarps][64];
-  __shared__ uint32_t pos_all[kRadWarps][64];  // (t << 20) | (h << 10) | w
   __shared__ uint32_t rbits_all[kRadWarps][kRadMaxWords];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = g.T;
@@ -63,59 +64,69 @@ __global__ void __launch_bounds__(kRadWarps * 32) radius_kernel(RadiusArgs a, Ge
   const int bh = int(row / g.nb), qb = int(row - long(bh) * g.nb);
   const float S = float(g.S);
 
-  // ---- the q-block's queries: position and squared base radius
-  float* r2 = r2_all[warp];
-  uint32_t* pos = pos_all[warp];
-  float r2max = 0.f;
-  for (int i = lane; i < 64; i += 32) {
-    const int tok = block_row_token(g, qb, i);
-    const int t = tok / (g.Hh * g.Ww), rem = tok - t * g.Hh * g.Ww;
-    const int h = rem / g.Ww, w = rem - h * g.Ww;
+  // ---- the q-block's queries (lane holds queries lane and lane + 32):
+  // position and squared base radius
+  int qtt[2], qhh[2], qww[2];
+  float r2q[2];
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int tok = block_row_token(g, qb, lane + 32 * u);
+    qtt[u] = tok / (g.Hh * g.Ww);
+    const int rem = tok - qtt[u] * g.Hh * g.Ww;
+    qhh[u] = rem / g.Ww;
+    qww[u] = rem - qhh[u] * g.Ww;
     const float H = a.entropy[size_t(bh) * g.S + tok];
     const float k = fminf(a.tau * expf(H), S);
-    r2[i] = k * zinv_tab[t];
-    pos[i] = (uint32_t(t) << 20) | (uint32_t(h) << 10) | uint32_t(w);
-    r2max = fmaxf(r2max, r2[i]);
+    r2q[u] = k * zinv_tab[qtt[u]];
   }
+  float r2max = fmaxf(r2q[0], r2q[1]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) r2max = fmaxf(r2max, __shfl_xor_sync(0xFFFFFFFFu, r2max, o));
-  __syncwarp();
   int qt, qh, qw;
   block_coords(g, qb, qt, qh, qw);
   const int qt0 = qt * g.pt, qt1 = qt0 + g.pt - 1;
   const int qh0 = qh * g.ph, qh1 = qh0 + g.ph - 1;
   const int qw0 = qw * g.pw, qw1 = qw0 + g.pw - 1;
 
-  // ---- votes per k-block, 32 k-blocks per round (lane = k-block)
+  // ---- votes per k-block: 32 k-blocks per round (lane = k-block) for the
+  // pruning test, then every unpruned one voted on by all 64 queries
   uint32_t* rbits = rbits_all[warp];
   const int nwords = bitmap_words(g);
   for (int base = 0; base < g.nb; base += 32) {
     const int kb = base + lane;
-    bool keep = false;
+    bool live = false;
+    uint32_t corner = 0u;  // (t0 << 20) | (h0 << 10) | w0 of the k-block's box
     if (kb < g.nb) {
       int kt, kh, kw;
       block_coords(g, kb, kt, kh, kw);
       const int kt0 = kt * g.pt, kt1 = kt0 + g.pt - 1;
       const int kh0 = kh * g.ph, kh1 = kh0 + g.ph - 1;
       const int kw0 = kw * g.pw, kw1 = kw0 + g.pw - 1;
+      corner = (uint32_t(kt0) << 20) | (uint32_t(kh0) << 10) | uint32_t(kw0);
       // prune: the nearest points of the two boxes, at the largest radius
       const int bt = kt0 > qt1 ? kt0 - qt1 : (qt0 > kt1 ? qt0 - kt1 : 0);
       const int bhd = kh0 > qh1 ? kh0 - qh1 : (qh0 > kh1 ? qh0 - kh1 : 0);
       const int bwd = kw0 > qw1 ? kw0 - qw1 : (qw0 > kw1 ? qw0 - kw1 : 0);
-      if (float(bhd * bhd + bwd * bwd) <= r2max * f_tab[bt]) {
-        int votes = 0;
-        for (int i = 0; i < 64 && votes < a.vote_min; ++i) {
-          const uint32_t p = pos[i];
-          const int t = int(p >> 20), h = int((p >> 10) & 1023u), w = int(p & 1023u);
-          const int dt = dist_to_range(t, kt0, kt1);
-          const int dh = dist_to_range(h, kh0, kh1), dw = dist_to_range(w, kw0, kw1);
-          votes += float(dh * dh + dw * dw) <= r2[i] * f_tab[dt] ? 1 : 0;
-        }
-        keep = votes >= a.vote_min;
-      }
+      live = float(bhd * bhd + bwd * bwd) <= r2max * f_tab[bt];
     }
-    const unsigned b = __ballot_sync(0xFFFFFFFFu, keep);
-    if (lane == 0) rbits[base >> 5] = b;
+    uint32_t unp = __ballot_sync(0xFFFFFFFFu, live), keep = 0u;
+    while (unp) {  // warp-uniform
+      const int j = __ffs(unp) - 1;
+      unp &= unp - 1u;
+      const uint32_t c = __shfl_sync(0xFFFFFFFFu, corner, j);
+      const int kt0 = int(c >> 20), kh0 = int((c >> 10) & 1023u), kw0 = int(c & 1023u);
+      const int kt1 = kt0 + g.pt - 1, kh1 = kh0 + g.ph - 1, kw1 = kw0 + g.pw - 1;
+      int votes = 0;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int dt = dist_to_range(qtt[u], kt0, kt1);
+        const int dh = dist_to_range(qhh[u], kh0, kh1), dw = dist_to_range(qww[u], kw0, kw1);
+        votes += __popc(__ballot_sync(0xFFFFFFFFu,
+                                      float(dh * dh + dw * dw) <= r2q[u] * f_tab[dt]));
+      }
+      if (votes >= a.vote_min) keep |= 1u << j;
+    }
+    if (lane == 0) rbits[base >> 5] = keep;
   }
   __syncwarp();
 
