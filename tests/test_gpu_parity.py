@@ -275,6 +275,22 @@ def test_edge_shapes(w):
     check_out_full(w, out, gm)
 
 
+# Rows of 1025 and 2048 blocks: the bounds of the select kernel that holds a
+# row in a pair of warps (at 1025 the second warp holds one column).
+PAIR_EDGE = [
+    W.HUNYUAN.with_(name="pair_lo_1x2x65600x128", H=2, T=41, Hh=40, Ww=40),
+    W.HUNYUAN.with_(name="pair_hi_1x1x131072x128_sta3", H=1, T=32, Hh=64, Ww=64, sta=(3, 3, 3)),
+]
+
+
+@pytest.mark.parametrize("w", PAIR_EDGE, ids=[e.name for e in PAIR_EDGE])
+def test_pair_select_bounds(w):
+    assert w.nb in (1025, 2048)
+    out, gm, views, desc, _ = run(w)
+    check_mask(w, gm)
+    check_out_qblocks(w, out, gm, views, desc, heads=(0,), per_head=8)
+
+
 def test_dense_threshold_matches_sdpa():
     w = W.W8K.with_(thr=0.0, sta=(0, 0, 0))
     out, gm, *_ = run(w, out_fp32=True)
